@@ -1,0 +1,231 @@
+/*
+ * sta.h -- C ABI of the sparse spatiotemporal attention library (libsta.so).
+ *
+ * Content-adaptive sparse self-attention over a video latent grid of
+ * F frames x H x W tokens, for B200 (sm_100a).  Two stages:
+ *
+ *   sta_build_blocks     selector: Q, K (or geometry) -> integer KV-unit lists
+ *   sta_sparse_attn_fwd  exact softmax attention over the kept units only
+ *   sta_dense_attn_fwd   the same kernel over every key (the denominator of
+ *                        the speedup metric)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors q, k, v, o are [heads][N][d], N = F*H*W, tokens in raster order
+ *   (frame-major, then row h, then column w), d contiguous.  Element type is
+ *   sta_problem.dtype (bf16, or fp32 which is rounded to bf16 on the device
+ *   before the tensor cores; o then is fp32).
+ * - Every pointer argument that names tensor data is a DEVICE pointer owned
+ *   by the caller.  The library never allocates, frees or retains memory and
+ *   keeps no state between calls.  Scratch space, where needed, is passed in
+ *   as `workspace` after querying its size.
+ * - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
+ *   legacy default stream) and returns.  Results are valid once the caller
+ *   has synchronised the stream.
+ * - The host return value reports argument errors and launch failures.
+ *   In-kernel errors are OR-ed into the caller's device word `dev_status`
+ *   (an int32 in device memory, may be NULL) as STA_DEV_* bits; decode it
+ *   after synchronising with sta_dev_status_string().
+ * - Shapes supported: d in {64, 128}; block_q in {16, 32, 64, 128};
+ *   kv_unit in {16, 32, 64, 128}.  Anything else returns STA_ERR_UNSUPPORTED.
+ *   There is no CPU path.
+ *
+ * Page references are to the pages this library restates:
+ *   [TRA]   "Token Radius Attention for Efficient Video Generation"
+ *   [RAD]   "Radial Attention to Accelerate Video Generation"
+ *   [HETA]  "Where Compute Matters: Heterogeneous Attention for Efficient
+ *            Video Diffusion"
+ *   [AB]    "AB-Attention speeds up video diffusion transformers up to 2.23x,
+ *            no training"
+ */
+#ifndef STA_H
+#define STA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (binary-compatible with cudaStream_t). */
+typedef struct CUstream_st* sta_stream_t;
+
+typedef enum {
+  STA_OK = 0,
+  STA_ERR_ARG = -1,          /* null pointer, bad dimension, inconsistent sizes */
+  STA_ERR_UNSUPPORTED = -2,  /* valid request outside the supported shapes     */
+  STA_ERR_CAPACITY = -3,     /* a list row needs more than `cap` entries       */
+  STA_ERR_CUDA = -4,         /* a CUDA runtime/driver call or launch failed    */
+  STA_ERR_WORKSPACE = -5     /* workspace pointer NULL or smaller than needed  */
+} sta_status;
+
+/* Bits OR-ed into *dev_status by kernels. */
+#define STA_DEV_TIMEOUT   0x1  /* a bounded wait ran out; the CTA abandoned its work */
+#define STA_DEV_CAPACITY  0x2  /* a list row was truncated at `cap`                  */
+#define STA_DEV_EMPTY_ROW 0x4  /* a query row had no kept key; its output is 0      */
+#define STA_DEV_BAD_INDEX 0x8  /* a list entry was out of range and was skipped     */
+
+typedef enum { STA_BF16 = 0, STA_F32 = 1 } sta_dtype;
+
+typedef enum {
+  STA_SEL_RADIAL = 0,    /* static radial window         [RAD] The idea behind Radial Attention */
+  STA_SEL_ENTROPY = 1,   /* pooled entropy -> radius     [TRA] 2. Methodology, The TRA Pipeline */
+  STA_SEL_IBCS_SIP = 2,  /* k-means importance + Philox inclusion-probability sampling  [AB]   */
+  STA_SEL_ROUTED = 3     /* difficulty routing: dense for the top fraction, local window [HETA] */
+} sta_selector;
+
+/* Problem geometry.  N = F*H*W tokens per head. */
+typedef struct {
+  int heads, F, H, W, d;
+  sta_dtype dtype;
+} sta_problem;
+
+/*
+ * Selector parameters.  Only the group of the chosen kind is read.
+ *
+ * radial   [RAD]: window at frame distance df (tokens):
+ *            w(df) = H*W                                  if df <= full_df
+ *                  = w0 >> floor(log2(df + w_off))         otherwise
+ *          query token i and key token j are related iff |s_i - s_j| < w(|f_i - f_j|)
+ *          (s = h*W + w inside a frame); a block pair is kept iff any of its
+ *          token pairs is related.  Lists are shared by all heads.
+ * entropy  [TRA]: pooled block means, H_b = entropy of softmax_c(Qbar_b.Kbar_c/sqrt(d)),
+ *          radius r_b = clamp(floor(alpha + beta*H_b), r_lo, r_hi) (fp32),
+ *          key block kept iff the Chebyshev distance of block cells
+ *          (f, h/tile_h, w/tile_w) of the blocks' centre tokens is <= r_b.
+ * ibcs_sip [AB]: k-means (km_k centroids, km_iters iterations) of each query
+ *          block's queries; importance p_j of kv_unit-token sub-blocks;
+ *          pi_j = min(1, lambda p_j), sum pi = ceil(sample_frac * n_sub);
+ *          keep j iff u_j < pi_j with u_j from Philox4x32-10 (key = seed,
+ *          counter = (j/4, 0, head*n_qblocks + qblock, 0)); logw_j = -ln pi_j.
+ * routed   [HETA]: the ceil(dense_frac*N) tokens of highest difficulty (fp32,
+ *          ties to the lower index) attend to all keys; every other token
+ *          attends to keys with |df| <= win_f, dh in [-win_h, win_h),
+ *          dw in [-win_w, win_w).  `difficulty` is a device pointer [N].
+ */
+typedef struct {
+  sta_selector kind;
+  int block_q;   /* query block size in tokens                          */
+  int kv_unit;   /* key/value unit size in tokens (list entries)        */
+  /* radial */
+  int radial_w0, radial_w_off, radial_full_df;
+  /* entropy */
+  float ent_alpha, ent_beta;
+  int ent_r_lo, ent_r_hi, ent_tile_h, ent_tile_w;
+  /* ibcs_sip */
+  int km_k, km_iters;
+  float sample_frac;
+  uint64_t seed;
+  /* routed */
+  float dense_frac;
+  int win_f, win_h, win_w;
+  const float* difficulty;
+} sta_selector_params;
+
+/*
+ * Block lists (ELL layout), all device memory owned by the caller.
+ *   rows      = n_qblocks (head_shared = 1) or heads * n_qblocks, with
+ *               n_qblocks = ceil(N / block_q)
+ *   idx       [rows][cap] int32 unit ids, ascending; unit u covers tokens
+ *             [u*kv_unit, min((u+1)*kv_unit, N))
+ *   cnt       [rows] int32 number of valid entries per row
+ *   logw      [rows][cap] float, -ln(pi) per entry (ibcs_sip) or NULL
+ *   required_cap  device int32, written with the largest row length seen
+ *             (may be NULL).  Rows longer than cap are truncated and
+ *             STA_DEV_CAPACITY is raised.
+ * Routed extras (STA_SEL_ROUTED; the local lists above then hold the
+ * kv_unit units touched by each query block's local windows):
+ *   routed_ids   [n_routed] int32 ascending routed token ids
+ *   routed_flag  [N] uint8, 1 if the token is routed
+ *   n_routed     host field, set by sta_build_blocks
+ * Entropy extras (STA_SEL_ENTROPY, optional):
+ *   entropy [heads][n_qblocks] float, radius [heads][n_qblocks] int32
+ */
+typedef struct {
+  int32_t* idx;
+  int32_t* cnt;
+  float* logw;
+  int32_t cap;
+  int32_t head_shared;
+  int32_t* required_cap;
+  int32_t* routed_ids;
+  uint8_t* routed_flag;
+  int32_t n_routed;
+  float* entropy;
+  int32_t* radius;
+} sta_block_lists;
+
+/* Workspace bytes sta_build_blocks needs for this problem and selector. */
+size_t sta_build_blocks_workspace(const sta_problem* prob, const sta_selector_params* sel);
+
+/* Rows of the lists the selector writes (n_qblocks, or heads*n_qblocks). */
+int sta_build_blocks_rows(const sta_problem* prob, const sta_selector_params* sel);
+
+/*
+ * Stage (a): selector.  q, k: device tensors [heads][N][d] (may be NULL for
+ * the radial and routed kinds, which read only geometry / difficulty).
+ * Writes `out` (see sta_block_lists).  Asynchronous on `stream`.
+ * Errors: STA_ERR_ARG (null/inconsistent), STA_ERR_UNSUPPORTED (shape),
+ * STA_ERR_WORKSPACE, STA_ERR_CUDA.
+ */
+sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* sel,
+                            const void* q, const void* k, sta_block_lists* out,
+                            void* workspace, size_t workspace_bytes,
+                            int32_t* dev_status, sta_stream_t stream);
+
+/* Attention modes. */
+typedef enum {
+  STA_ATTN_LISTS = 0,   /* per (head, query block) rows of `lists`                  */
+  STA_ATTN_ROUTED = 1   /* routed rows dense over all keys + local lists w/ window  */
+} sta_attn_mode;
+
+typedef struct {
+  sta_attn_mode mode;
+  int block_q;       /* query block of the lists (tokens)                   */
+  int kv_unit;       /* unit size of the list entries (tokens)              */
+  float scale;       /* logit scale; <= 0 selects 1/sqrt(d)                 */
+  int win_f, win_h, win_w;  /* STA_ATTN_ROUTED local window                 */
+} sta_attn_params;
+
+/* Workspace bytes of the attention calls (0 for bf16 inputs). */
+size_t sta_attn_workspace(const sta_problem* prob);
+
+/*
+ * Stage (b): exact attention over the kept units.
+ * [TRA] 1. Problem Statement (block-level sparsity) and The TRA Pipeline;
+ * [AB] method paragraph (pruned blocks vanish from the softmax; sampled
+ * units weighted by 1/pi; small units packed into full tensor-core tiles).
+ * For query i with kept key set K_i and weights w (1, or exp(logw)):
+ *   O_i = sum_k w_k exp(s_ik - m_i) v_k / sum_k w_k exp(s_ik - m_i),
+ *   s_ik = scale * q_i.k_k.  Rows with no kept key get O_i = 0.
+ * o: device [heads][N][d] (bf16, or fp32 when dtype is STA_F32).  Rows not
+ * covered by any list row are left untouched.
+ */
+sta_status sta_sparse_attn_fwd(const sta_problem* prob, const sta_attn_params* prm,
+                               const void* q, const void* k, const void* v,
+                               const sta_block_lists* lists, void* o,
+                               void* workspace, size_t workspace_bytes,
+                               int32_t* dev_status, sta_stream_t stream);
+
+/*
+ * Dense softmax attention over all N keys ([TRA] 1. Problem Statement),
+ * the same kernel with an implicit full list of 128-key units.
+ */
+sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void* k,
+                              const void* v, float scale, void* o,
+                              void* workspace, size_t workspace_bytes,
+                              int32_t* dev_status, sta_stream_t stream);
+
+/* Static description of a status code / of the device status bits. */
+const char* sta_status_string(sta_status s);
+const char* sta_dev_status_string(int32_t bits);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int sta_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STA_H */

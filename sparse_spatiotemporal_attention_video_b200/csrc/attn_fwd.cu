@@ -1,0 +1,698 @@
+// attn_fwd.cu -- exact block-sparse softmax attention on sm_100a.
+//
+// What it computes ("Token Radius Attention for Efficient Video Generation",
+// 1. Problem Statement and The TRA Pipeline; "AB-Attention ..." method
+// paragraph): for every query row i of a work item and the key units listed
+// for it, O_i = sum_k w_k exp(s_ik - m_i) v_k / sum_k w_k exp(s_ik - m_i)
+// with s_ik = scale * q_i.k_k; keys outside the listed units never enter the
+// softmax; w_k = 1/pi of the key's sampled unit (stored as -ln pi) or 1.
+//
+// How (one persistent CTA per SM, 6 warps):
+//   warp 0      producer: TMA loads of the 128-row Q tile and, per 128-key
+//               tile, of the listed key/value units (kv_unit rows each,
+//               128-byte swizzle) into a K ring and a V ring; gathered query
+//               rows (routed items) are copied by the warp and swizzled by
+//               hand.
+//   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM
+//               S buffers (tcgen05.mma, M=128 N=128 K=16 steps, both
+//               operands K-major in shared memory), then O += P V with P
+//               read from TMEM (bf16, aliased onto the S buffer) and V
+//               MN-major in shared memory.  QK of tile t+1 is issued before
+//               PV of tile t, so the tensor core works on the next tile while
+//               the softmax warps handle the current one.
+//   warps 2-5   softmax: thread r owns query row r (TMEM lane r): loads its
+//               128 logits, masks partial units / window, adds log-weights,
+//               keeps a running max and sum in registers (max updates that
+//               move by <= 8 in log2 units are deferred, so O in TMEM is
+//               rescaled only on large jumps), writes P as bf16 into TMEM,
+//               and finally normalises O and stores it.
+// Every wait is bounded; a timeout raises STA_DEV_TIMEOUT, sets a CTA-wide
+// abort flag and unwinds without trapping.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace sta {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kHalfBytes = 128 * 128;  // 128 rows x 128 bytes: one 64-column half of a tile
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D, int KS, int VS>
+struct Layout {
+  static constexpr int DH = D / 64;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
+  // barriers: q_full, q_empty, k_full[KS], k_empty[KS], v_full[VS],
+  // v_empty[VS], s_full[2], p_full[2], o_done[2], mma_done
+  static constexpr int NBAR = 2 + 2 * KS + 2 * VS + 7;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024
+};
+
+struct Item {
+  int head, kind, q_start, q_len, row, gbase, ntiles, unit, upt;
+};
+
+__device__ __forceinline__ Item decode_item(const AttnArgs& a, int it) {
+  Item I;
+  I.gbase = 0;
+  I.row = -1;
+  if (a.mode == kModeRouted) {
+    const int nd = a.heads * a.n_dense_items;
+    if (it < nd) {
+      I.head = it / a.n_dense_items;
+      const int j = it - I.head * a.n_dense_items;
+      I.kind = kItemGatherDense;
+      I.gbase = j * kTileQ;
+      I.q_start = 0;
+      I.q_len = min(kTileQ, a.n_routed - I.gbase);
+      I.unit = kTileK;
+      I.upt = 1;
+      I.ntiles = (a.N + kTileK - 1) / kTileK;
+      return I;
+    }
+    it -= nd;
+    I.kind = kItemLocal;
+  } else {
+    I.kind = (a.mode == kModeDense) ? kItemDense : kItemList;
+  }
+  I.head = it / a.n_qb;
+  const int qb = it - I.head * a.n_qb;
+  I.q_start = qb * a.block_q;
+  I.q_len = min(a.block_q, a.N - I.q_start);
+  if (I.kind == kItemDense) {
+    I.unit = kTileK;
+    I.upt = 1;
+    I.ntiles = (a.N + kTileK - 1) / kTileK;
+  } else {
+    I.row = a.head_shared ? qb : I.head * a.n_qb + qb;
+    I.unit = a.unit;
+    I.upt = kTileK / a.unit;
+    int c = __ldg(a.cnt + I.row);
+    c = max(0, min(c, a.cap));
+    I.ntiles = (c + I.upt - 1) / I.upt;
+  }
+  return I;
+}
+
+// Unit loaded into slot s of tile t of item I.  Returns the unit id to load
+// (always a valid unit), the number of valid keys in the slot (0 for an
+// empty slot or a bad list entry) and the entry's log-weight.
+__device__ __forceinline__ int slot_unit(const AttnArgs& a, const Item& I, int t, int s,
+                                         int& nvalid, float& lw, bool& bad) {
+  lw = 0.f;
+  bad = false;
+  if (I.kind == kItemDense || I.kind == kItemGatherDense) {
+    nvalid = min(kTileK, a.N - t * kTileK);
+    return t;
+  }
+  const int pos = t * I.upt + s;
+  int c = __ldg(a.cnt + I.row);
+  c = max(0, min(c, a.cap));
+  if (pos >= c) {
+    nvalid = 0;
+    return 0;
+  }
+  const size_t off = static_cast<size_t>(I.row) * a.cap + pos;
+  const int u = __ldg(a.idx + off);
+  const int n_units = (a.N + I.unit - 1) / I.unit;
+  if (u < 0 || u >= n_units) {
+    nvalid = 0;
+    bad = true;
+    return 0;
+  }
+  nvalid = min(I.unit, a.N - u * I.unit);
+  if (a.logw) lw = __ldg(a.logw + off);
+  return u;
+}
+
+__device__ __forceinline__ void fail(volatile int* abort, int32_t* st) {
+  *abort = 1;
+  raise_status(st, STA_DEV_TIMEOUT);
+}
+
+// Per-slot information of one tile for the softmax threads.
+template <int UNIT>
+struct TileInfo {
+  static constexpr int UPT = kTileK / UNIT;
+  int nv[UPT];
+  float braw[UPT];   // log-weight / scale: added to raw logits
+  int base[UPT];     // first token of the unit
+  bool full, bias;
+};
+
+template <int UNIT>
+__device__ __forceinline__ void load_tile_info(const AttnArgs& a, const Item& I, int t,
+                                               float inv_scale, TileInfo<UNIT>& ti) {
+  ti.full = true;
+  ti.bias = (a.logw != nullptr) && (I.kind == kItemList || I.kind == kItemLocal);
+#pragma unroll
+  for (int s = 0; s < TileInfo<UNIT>::UPT; ++s) {
+    int nv;
+    float lw;
+    bool bad;
+    const int u = slot_unit(a, I, t, s, nv, lw, bad);
+    ti.nv[s] = nv;
+    ti.braw[s] = lw * inv_scale;
+    ti.base[s] = u * UNIT;
+    if (nv < UNIT) ti.full = false;
+  }
+}
+
+// Raw logits of one thread's row -> masked/biased raw logits in place.
+template <int UNIT>
+__device__ __forceinline__ void mask_and_bias(float (&x)[128], const TileInfo<UNIT>& ti,
+                                              bool window, const AttnArgs& a, int fq, int hq,
+                                              int wq) {
+  constexpr int UPT = TileInfo<UNIT>::UPT;
+  if (!ti.full) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c) {
+      if ((c % UNIT) >= ti.nv[c / UNIT]) x[c] = -INFINITY;
+    }
+  }
+  if (ti.bias) {
+#pragma unroll
+    for (int c = 0; c < 128; ++c) x[c] += ti.braw[c / UNIT];
+  }
+  if (window) {
+    const int S = a.H * a.W;
+#pragma unroll
+    for (int s = 0; s < UPT; ++s) {
+      const int t0 = ti.base[s];
+      int f = t0 / S;
+      int rem = t0 - f * S;
+      int h = rem / a.W;
+      int w = rem - h * a.W;
+#pragma unroll
+      for (int e = 0; e < UNIT; ++e) {
+        const int c = s * UNIT + e;
+        const int df = f - fq, dh = h - hq, dw = w - wq;
+        const bool in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
+                        (dh < a.win_h) && (dw >= -a.win_w) && (dw < a.win_w);
+        if (!in) x[c] = -INFINITY;
+        if (++w == a.W) {
+          w = 0;
+          if (++h == a.H) {
+            h = 0;
+            ++f;
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int D, int KS, int VS, int UNIT>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k_u,
+                    const __grid_constant__ CUtensorMap tm_v_u,
+                    const __grid_constant__ CUtensorMap tm_k_f,
+                    const __grid_constant__ CUtensorMap tm_v_f) {
+  using L = Layout<D, KS, VS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  uint8_t* sQ = smem + L::OFF_Q;
+  uint8_t* sK = smem + L::OFF_K;
+  uint8_t* sV = smem + L::OFF_V;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* k_full = bars + 2;
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* s_full = v_empty + VS;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* mma_done = o_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int i = 0; i < KS; ++i) {
+      mbar_init(k_full + i, 1);
+      mbar_init(k_empty + i, 1);
+    }
+    for (int i = 0; i < VS; ++i) {
+      mbar_init(v_full + i, 1);
+      mbar_init(v_empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(s_full + i, 1);
+      mbar_init(p_full + i, 128);
+      mbar_init(o_done + i, 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k_u);
+    tma_prefetch_desc(&tm_v_u);
+    tma_prefetch_desc(&tm_k_f);
+    tma_prefetch_desc(&tm_v_f);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t limit = kWaitLimitNs;
+  int dummy_abort_storage = 0;
+  volatile int* no_abort = &dummy_abort_storage;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    uint32_t kt = 0, vt = 0, qn = 0;
+    for (int it = blockIdx.x; it < a.n_items; it += gridDim.x) {
+      if (*abort) break;
+      const Item I = decode_item(a, it);
+      if (I.ntiles == 0) continue;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(q_empty, (qn & 1) ^ 1, abort, limit);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) fail(abort, a.dev_status);
+        break;
+      }
+      if (I.kind == kItemGatherDense) {
+        // Gather the routed query rows and store them in the 128-byte
+        // swizzled layout TMA would produce (16-byte chunk c of row r sits
+        // at chunk c ^ (r % 8) of the row).
+        const __nv_bfloat16* qh = a.q + static_cast<size_t>(I.head) * a.N * D;
+        for (int r = lane; r < kTileQ; r += 32) {
+          const int src_r = (r < I.q_len) ? r : 0;
+          const int tok = __ldg(a.routed_ids + I.gbase + src_r);
+          const uint4* src = reinterpret_cast<const uint4*>(qh + static_cast<size_t>(tok) * D);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) {
+            const int h = c >> 3, cc = c & 7;
+            uint4 val = __ldg(src + c);
+            *reinterpret_cast<uint4*>(sQ + h * kHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = val;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_full);
+      } else if (lane == 0) {
+        mbar_arrive_expect_tx(q_full, L::TILE_BYTES);
+#pragma unroll
+        for (int h = 0; h < L::DH; ++h)
+          tma_load_3d(sQ + h * kHalfBytes, &tm_q, q_full, h * 64, I.q_start, I.head);
+      }
+      ++qn;
+      const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
+      const CUtensorMap* mk = dense_like ? &tm_k_f : &tm_k_u;
+      const CUtensorMap* mv = dense_like ? &tm_v_f : &tm_v_u;
+      const int unit = I.unit;
+      const int nops = I.upt * L::DH;
+      for (int t = 0; t < I.ntiles; ++t) {
+        // one lane per (slot, half) copy
+        int u = 0;
+        const int s = lane / L::DH, h = lane % L::DH;
+        if (lane < nops) {
+          int nv;
+          float lw;
+          bool bad;
+          u = slot_unit(a, I, t, s, nv, lw, bad);
+          if (bad) raise_status(a.dev_status, STA_DEV_BAD_INDEX);
+        }
+        // K
+        {
+          const int st = kt % KS;
+          if (lane == 0) ok = mbar_wait(k_empty + st, ((kt / KS) & 1) ^ 1, abort, limit);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          if (lane == 0) mbar_arrive_expect_tx(k_full + st, L::TILE_BYTES);
+          __syncwarp();
+          if (lane < nops)
+            tma_load_3d(sK + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mk,
+                        k_full + st, h * 64, u * unit, I.head);
+          ++kt;
+        }
+        // V
+        {
+          const int st = vt % VS;
+          if (lane == 0) ok = mbar_wait(v_empty + st, ((vt / VS) & 1) ^ 1, abort, limit);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          if (lane == 0) mbar_arrive_expect_tx(v_full + st, L::TILE_BYTES);
+          __syncwarp();
+          if (lane < nops)
+            tma_load_3d(sV + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mv,
+                        v_full + st, h * 64, u * unit, I.head);
+          ++vt;
+        }
+      }
+      if (!ok) {
+        if (lane == 0) fail(abort, a.dev_status);
+        break;
+      }
+    }
+    // Let every copy this warp issued land before the CTA can exit.
+    if (lane == 0) {
+      for (uint32_t i = (kt > KS ? kt - KS : 0); i < kt; ++i)
+        mbar_wait(k_full + (i % KS), (i / KS) & 1, no_abort, limit);
+      for (uint32_t i = (vt > VS ? vt - VS : 0); i < vt; ++i)
+        mbar_wait(v_full + (i % VS), (i / VS) & 1, no_abort, limit);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+      uint32_t kt = 0, vt = 0, qn = 0, g = 0;
+      bool ok = true;
+      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+        const uint32_t sb = gg & 1;
+        if (!mbar_wait(p_full + sb, (gg >> 1) & 1, abort, limit)) return false;
+        tc_fence_after();
+        const int st = vt % VS;
+        if (!mbar_wait(v_full + st, (vt / VS) & 1, abort, limit)) return false;
+        tc_fence_after();
+        const uint32_t tS = sb ? tS1 : tS0;
+        const uint32_t vbase = aV + st * L::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kTileK / 16; ++kk) {
+          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024);
+          mma_bf16_ts(tO, tS + kk * 8, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(v_empty + st);
+        ++vt;
+        mma_commit(o_done + sb);
+        return true;
+      };
+      for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
+        if (*abort) break;
+        const Item I = decode_item(a, it);
+        if (I.ntiles == 0) continue;
+        if (!mbar_wait(q_full, qn & 1, abort, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int t = 0; t < I.ntiles; ++t) {
+          const int st = kt % KS;
+          if (!mbar_wait(k_full + st, (kt / KS) & 1, abort, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = (g + t) & 1;
+          const uint32_t tS = sb ? tS1 : tS0;
+          const uint32_t kbase = aK + st * L::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+            const uint64_t adesc = smem_desc_sw128(aQ + off, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(kbase + off, 16, 1024);
+            mma_bf16_ss(tS, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(k_empty + st);
+          ++kt;
+          mma_commit(s_full + sb);
+          if (t == I.ntiles - 1) mma_commit(q_empty);
+          if (t > 0 && !issue_pv(g + t - 1, t == 1)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok) break;
+        if (!issue_pv(g + I.ntiles - 1, I.ntiles == 1)) {
+          ok = false;
+          break;
+        }
+        ++qn;
+        g += I.ntiles;
+      }
+      if (!ok) fail(abort, a.dev_status);
+      // all issued MMAs complete before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, no_abort, limit);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const float scale_log2 = a.scale_log2;
+    const float inv_scale = kLog2e / scale_log2;  // natural-log weight -> raw logit units
+    uint32_t g = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
+      if (*abort) break;
+      const Item I = decode_item(a, it);
+      int tok = -1;
+      if (I.kind == kItemGatherDense) {
+        if (r < I.q_len) tok = __ldg(a.routed_ids + I.gbase + r);
+      } else if (r < I.q_len) {
+        tok = I.q_start + r;
+      }
+      bool active = tok >= 0;
+      if (active && I.kind == kItemLocal && __ldg(a.routed_flag + tok)) active = false;
+      const size_t orow = static_cast<size_t>(I.head) * a.N + (tok < 0 ? 0 : tok);
+      if (I.ntiles == 0) {
+        if (active) {
+          if (a.out_f32) {
+            float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D);
+            for (int i = 0; i < D / 4; ++i) op[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          } else {
+            uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D);
+            for (int i = 0; i < D / 8; ++i) op[i] = make_uint4(0, 0, 0, 0);
+          }
+          raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
+        }
+        continue;
+      }
+      int fq = 0, hq = 0, wq = 0;
+      const bool window = (I.kind == kItemLocal);
+      if (window && tok >= 0) {
+        const int S = a.H * a.W;
+        fq = tok / S;
+        const int rem = tok - fq * S;
+        hq = rem / a.W;
+        wq = rem - hq * a.W;
+      }
+      const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int t = 0; t < I.ntiles; ++t) {
+        const uint32_t gg = g + t;
+        const uint32_t sb = gg & 1;
+        if (!mbar_wait(s_full + sb, (gg >> 1) & 1, abort, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        float x[128];
+        {
+          uint32_t v[32];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            tmem_ld32(tmem + lane_off + sb * 128 + j * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[j * 32 + i] = __uint_as_float(v[i]);
+          }
+        }
+        if (dense_like) {
+          TileInfo<kTileK> ti;
+          load_tile_info<kTileK>(a, I, t, inv_scale, ti);
+          mask_and_bias<kTileK>(x, ti, false, a, 0, 0, 0);
+        } else {
+          TileInfo<UNIT> ti;
+          load_tile_info<UNIT>(a, I, t, inv_scale, ti);
+          mask_and_bias<UNIT>(x, ti, window, a, fq, hq, wq);
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+        const float m_tile = mx * scale_log2;  // -inf if all masked
+        const float m_new = fmaxf(m_run, m_tile);
+        const bool need = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
+        if (__any_sync(0xffffffffu, need)) {
+          // O of this warp's rows holds tiles < t; the last of them must be
+          // accumulated before it is rescaled.
+          const uint32_t gp = gg - 1;
+          if (!mbar_wait(o_done + (gp & 1), (gp >> 1) & 1, abort, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = need ? fast_exp2(m_run - m_new) : 1.f;
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + 256 + ch * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+            tmem_st32(tmem + lane_off + 256 + ch * 32, v);
+          }
+          tmem_wait_st();
+          if (need) {
+            l_run *= f;
+            m_run = m_new;
+          }
+        }
+        if (m_run == -INFINITY) m_run = m_new;
+        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+        float lsum = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = fast_exp2(fmaf(x[c], scale_log2, -m_use));
+          const float p1 = fast_exp2(fmaf(x[c + 1], scale_log2, -m_use));
+          lsum += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+        l_run += lsum;
+        {
+          uint32_t v[32];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = pk[j * 32 + i];
+            tmem_st32(tmem + lane_off + sb * 128 + j * 32, v);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full + sb);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      const uint32_t gl = g + I.ntiles - 1;
+      if (!mbar_wait(o_done + (gl & 1), (gl >> 1) & 1, abort, limit)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      g += I.ntiles;
+      const bool empty = !(l_run > 0.f);
+      const float inv_l = empty ? 0.f : 1.f / l_run;
+      if (active && empty) raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
+#pragma unroll
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + 256 + ch * 32, v);
+        tmem_wait_ld();
+        if (active) {
+          if (a.out_f32) {
+            float4* op =
+                reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D + ch * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              op[i] = make_float4(__uint_as_float(v[4 * i]) * inv_l,
+                                  __uint_as_float(v[4 * i + 1]) * inv_l,
+                                  __uint_as_float(v[4 * i + 2]) * inv_l,
+                                  __uint_as_float(v[4 * i + 3]) * inv_l);
+          } else {
+            uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D +
+                                                 ch * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              op[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]) * inv_l,
+                                             __uint_as_float(v[8 * i + 1]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l,
+                                             __uint_as_float(v[8 * i + 3]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l,
+                                             __uint_as_float(v[8 * i + 5]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l,
+                                             __uint_as_float(v[8 * i + 7]) * inv_l));
+          }
+        }
+      }
+      tc_fence_before();
+    }
+    if (!ok) fail(abort, a.dev_status);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+__global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __restrict__ dst,
+                                   size_t n4) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = src[i];
+    dst[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+  }
+}
+
+template <int D, int KS, int VS, int UNIT>
+cudaError_t launch_t(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tku,
+                     const CUtensorMap& tvu, const CUtensorMap& tkf, const CUtensorMap& tvf,
+                     int num_sms, cudaStream_t stream) {
+  using L = Layout<D, KS, VS>;
+  auto kern = attn_fwd_kernel<D, KS, VS, UNIT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  if (e != cudaSuccess) return e;
+  const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kThreads, L::ALLOC, stream>>>(a, tq, tku, tvu, tkf, tvf);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tq,
+                             const CUtensorMap& tku, const CUtensorMap& tvu,
+                             const CUtensorMap& tkf, const CUtensorMap& tvf, int num_sms,
+                             cudaStream_t stream) {
+#define STA_ATTN_CASE(DD, UU)                                                                \
+  if (d == DD && a.unit == UU)                                                               \
+    return launch_t<DD, 2, 2, UU>(a, tq, tku, tvu, tkf, tvf, num_sms, stream);
+  STA_ATTN_CASE(128, 128)
+  STA_ATTN_CASE(128, 64)
+  STA_ATTN_CASE(128, 32)
+  STA_ATTN_CASE(128, 16)
+  STA_ATTN_CASE(64, 128)
+  STA_ATTN_CASE(64, 64)
+  STA_ATTN_CASE(64, 32)
+  STA_ATTN_CASE(64, 16)
+#undef STA_ATTN_CASE
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s) {
+  if (n % 4 != 0) return cudaErrorInvalidValue;
+  const size_t n4 = n / 4;
+  const int block = 256;
+  size_t grid = (n4 + block - 1) / block;
+  if (grid > 148 * 16) grid = 148 * 16;
+  if (grid == 0) return cudaSuccess;
+  f32_to_bf16_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(
+      reinterpret_cast<const float4*>(src), reinterpret_cast<uint2*>(dst), n4);
+  return cudaGetLastError();
+}
+
+}  // namespace sta

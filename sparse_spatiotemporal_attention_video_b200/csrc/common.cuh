@@ -1,0 +1,72 @@
+// common.cuh -- internal declarations shared by the library's translation
+// units (not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/sta.h"
+
+namespace sta {
+
+// Key/value tile width and query tile height of the attention kernel.
+constexpr int kTileQ = 128;
+constexpr int kTileK = 128;
+
+// Bounded-wait budget of every in-kernel wait (global-timer nanoseconds).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ void raise_status(int32_t* dev_status, int32_t bits) {
+  if (dev_status) atomicOr(dev_status, bits);
+}
+
+enum AttnKind : int {
+  kItemList = 0,       // raster query block, keys from a list row
+  kItemDense = 1,      // raster query block, every key
+  kItemGatherDense = 2,  // gathered (routed) query rows, every key
+  kItemLocal = 3       // raster query block, list row + local window predicate
+};
+
+enum AttnMode : int { kModeLists = 0, kModeDense = 1, kModeRouted = 2 };
+
+struct AttnArgs {
+  int heads, N, F, H, W;
+  float scale_log2;  // logit scale * log2(e)
+  int mode;
+  int block_q;       // raster query block (tokens)
+  int unit;          // list unit size (tokens)
+  int n_qb;          // ceil(N / block_q)
+  int n_items;
+  // lists
+  const int32_t* idx;
+  const int32_t* cnt;
+  const float* logw;
+  int cap;
+  int head_shared;
+  // routed
+  const int32_t* routed_ids;
+  const uint8_t* routed_flag;
+  int n_routed;
+  int n_dense_items;  // per head = ceil(n_routed / kTileQ)
+  int win_f, win_h, win_w;
+  // tensors
+  const __nv_bfloat16* q;  // for gathered query rows
+  void* o;
+  int out_f32;
+  int32_t* dev_status;
+};
+
+// Launchers (attn_fwd.cu).
+cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tm_q,
+                             const CUtensorMap& tm_k_unit, const CUtensorMap& tm_v_unit,
+                             const CUtensorMap& tm_k_full, const CUtensorMap& tm_v_full,
+                             int num_sms, cudaStream_t stream);
+cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
+
+// Radial selector (sel_radial.cu).
+cudaError_t launch_radial_lists(int F, int H, int W, int B, int w0, int w_off, int full_df,
+                                int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
+                                int32_t* dev_status, cudaStream_t stream);
+
+}  // namespace sta

@@ -1,0 +1,291 @@
+// sta_api.cu -- the C ABI (include/sta.h): argument checks, tensor-map
+// construction and kernel dispatch.  Every entry point only enqueues work
+// on the caller's stream; nothing here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+using namespace sta;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3D map over a [heads][N][d] bf16 tensor: dim0 = d (contiguous), dim1 = N,
+// dim2 = heads; box = 64 columns (128 bytes, 128-byte swizzle) x rows x 1.
+// Rows past N read as zero.
+bool make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                           static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool pow2_unit(int u) { return u == 16 || u == 32 || u == 64 || u == 128; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+sta_status check_problem(const sta_problem* p) {
+  if (!p) return STA_ERR_ARG;
+  if (p->heads < 1 || p->F < 1 || p->H < 1 || p->W < 1) return STA_ERR_ARG;
+  if (p->dtype != STA_BF16 && p->dtype != STA_F32) return STA_ERR_ARG;
+  if (p->d != 64 && p->d != 128) return STA_ERR_UNSUPPORTED;
+  const long long N = static_cast<long long>(p->F) * p->H * p->W;
+  if (N > (1ll << 30)) return STA_ERR_UNSUPPORTED;
+  if (N * p->heads > (1ll << 31) - 1) return STA_ERR_UNSUPPORTED;
+  return STA_OK;
+}
+
+int num_sms_current() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+size_t staged_bytes(const sta_problem* p) {
+  const size_t n = static_cast<size_t>(p->heads) * p->F * p->H * p->W * p->d;
+  return round_up(n * 2, 256);
+}
+
+// bf16 views of q, k, v: the inputs themselves, or fp32 inputs rounded
+// into the workspace.
+sta_status stage_inputs(const sta_problem* p, const void* q, const void* k, const void* v,
+                        void* ws, size_t ws_bytes, const __nv_bfloat16** qb,
+                        const __nv_bfloat16** kb, const __nv_bfloat16** vb,
+                        cudaStream_t stream) {
+  if (p->dtype == STA_BF16) {
+    *qb = static_cast<const __nv_bfloat16*>(q);
+    *kb = static_cast<const __nv_bfloat16*>(k);
+    *vb = static_cast<const __nv_bfloat16*>(v);
+    return STA_OK;
+  }
+  const size_t one = staged_bytes(p);
+  if (!ws || ws_bytes < 3 * one) return STA_ERR_WORKSPACE;
+  const size_t n = static_cast<size_t>(p->heads) * p->F * p->H * p->W * p->d;
+  __nv_bfloat16* base = static_cast<__nv_bfloat16*>(ws);
+  __nv_bfloat16* dq = base;
+  __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(ws) + one);
+  __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(ws) + 2 * one);
+  if (launch_f32_to_bf16(static_cast<const float*>(q), dq, n, stream) != cudaSuccess ||
+      launch_f32_to_bf16(static_cast<const float*>(k), dk, n, stream) != cudaSuccess ||
+      launch_f32_to_bf16(static_cast<const float*>(v), dv, n, stream) != cudaSuccess)
+    return STA_ERR_CUDA;
+  *qb = dq;
+  *kb = dk;
+  *vb = dv;
+  return STA_OK;
+}
+
+sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16* qb,
+                         const __nv_bfloat16* kb, const __nv_bfloat16* vb, int unit,
+                         cudaStream_t stream) {
+  CUtensorMap tq, tku, tvu, tkf, tvf;
+  const int N = a.N;
+  if (!make_map(&tq, qb, p->d, N, p->heads, kTileQ) ||
+      !make_map(&tku, kb, p->d, N, p->heads, unit) ||
+      !make_map(&tvu, vb, p->d, N, p->heads, unit) ||
+      !make_map(&tkf, kb, p->d, N, p->heads, kTileK) ||
+      !make_map(&tvf, vb, p->d, N, p->heads, kTileK))
+    return STA_ERR_CUDA;
+  const int sms = num_sms_current();
+  if (sms <= 0) return STA_ERR_CUDA;
+  a.unit = unit;
+  a.q = qb;
+  if (launch_attention(p->d, a, tq, tku, tvu, tkf, tvf, sms, stream) != cudaSuccess)
+    return STA_ERR_CUDA;
+  return STA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sta_version(void) { return kVersion; }
+
+const char* sta_status_string(sta_status s) {
+  switch (s) {
+    case STA_OK: return "ok";
+    case STA_ERR_ARG: return "invalid argument";
+    case STA_ERR_UNSUPPORTED: return "unsupported shape or parameter";
+    case STA_ERR_CAPACITY: return "list capacity exceeded";
+    case STA_ERR_CUDA: return "CUDA error";
+    case STA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char* sta_dev_status_string(int32_t bits) {
+  if (bits == 0) return "ok";
+  if (bits & STA_DEV_TIMEOUT) return "timeout: a bounded wait ran out";
+  if (bits & STA_DEV_BAD_INDEX) return "list entry out of range (skipped)";
+  if (bits & STA_DEV_CAPACITY) return "list row truncated at capacity";
+  if (bits & STA_DEV_EMPTY_ROW) return "query row without kept keys (output 0)";
+  return "unknown device status";
+}
+
+int sta_build_blocks_rows(const sta_problem* prob, const sta_selector_params* sel) {
+  if (check_problem(prob) != STA_OK || !sel || sel->block_q < 1) return -1;
+  const long long N = static_cast<long long>(prob->F) * prob->H * prob->W;
+  const int nqb = static_cast<int>((N + sel->block_q - 1) / sel->block_q);
+  switch (sel->kind) {
+    case STA_SEL_RADIAL:
+    case STA_SEL_ROUTED:
+      return nqb;
+    case STA_SEL_ENTROPY:
+    case STA_SEL_IBCS_SIP:
+      return nqb * prob->heads;
+  }
+  return -1;
+}
+
+size_t sta_build_blocks_workspace(const sta_problem* prob, const sta_selector_params* sel) {
+  if (check_problem(prob) != STA_OK || !sel) return 0;
+  return 0;
+}
+
+sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* sel,
+                            const void* q, const void* k, sta_block_lists* out, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  (void)q;
+  (void)k;
+  (void)workspace;
+  (void)workspace_bytes;
+  sta_status st = check_problem(prob);
+  if (st != STA_OK) return st;
+  if (!sel || !out || !out->idx || !out->cnt || out->cap < 1) return STA_ERR_ARG;
+  if (!pow2_unit(sel->block_q) || !pow2_unit(sel->kv_unit)) return STA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (sel->kind) {
+    case STA_SEL_RADIAL: {
+      if (sel->kv_unit != sel->block_q) return STA_ERR_UNSUPPORTED;
+      const int S = prob->H * prob->W;
+      if ((sel->block_q + S - 1) / S + 1 > 8) return STA_ERR_UNSUPPORTED;
+      out->head_shared = 1;
+      if (launch_radial_lists(prob->F, prob->H, prob->W, sel->block_q, sel->radial_w0,
+                              sel->radial_w_off, sel->radial_full_df, out->idx, out->cnt, out->cap,
+                              out->required_cap, dev_status, s) != cudaSuccess)
+        return STA_ERR_CUDA;
+      return STA_OK;
+    }
+    default:
+      return STA_ERR_UNSUPPORTED;
+  }
+}
+
+size_t sta_attn_workspace(const sta_problem* prob) {
+  if (check_problem(prob) != STA_OK) return 0;
+  return prob->dtype == STA_F32 ? 3 * staged_bytes(prob) : 0;
+}
+
+sta_status sta_sparse_attn_fwd(const sta_problem* prob, const sta_attn_params* prm,
+                               const void* q, const void* k, const void* v,
+                               const sta_block_lists* lists, void* o, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  sta_status st = check_problem(prob);
+  if (st != STA_OK) return st;
+  if (!prm || !q || !k || !v || !lists || !o) return STA_ERR_ARG;
+  if (!pow2_unit(prm->block_q) || !pow2_unit(prm->kv_unit)) return STA_ERR_UNSUPPORTED;
+  if (!lists->idx || !lists->cnt || lists->cap < 1) return STA_ERR_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int N = prob->F * prob->H * prob->W;
+  AttnArgs a = {};
+  a.heads = prob->heads;
+  a.N = N;
+  a.F = prob->F;
+  a.H = prob->H;
+  a.W = prob->W;
+  const float scale = prm->scale > 0.f ? prm->scale : 1.0f / sqrtf(static_cast<float>(prob->d));
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.block_q = prm->block_q;
+  a.n_qb = (N + prm->block_q - 1) / prm->block_q;
+  a.idx = lists->idx;
+  a.cnt = lists->cnt;
+  a.logw = lists->logw;
+  a.cap = lists->cap;
+  a.head_shared = lists->head_shared ? 1 : 0;
+  a.o = o;
+  a.out_f32 = prob->dtype == STA_F32;
+  a.dev_status = dev_status;
+  if (prm->mode == STA_ATTN_LISTS) {
+    a.mode = kModeLists;
+    a.n_items = prob->heads * a.n_qb;
+  } else if (prm->mode == STA_ATTN_ROUTED) {
+    if (!lists->routed_ids || !lists->routed_flag || lists->n_routed < 0 || lists->n_routed > N)
+      return STA_ERR_ARG;
+    if (!lists->head_shared) return STA_ERR_UNSUPPORTED;
+    a.mode = kModeRouted;
+    a.routed_ids = lists->routed_ids;
+    a.routed_flag = lists->routed_flag;
+    a.n_routed = lists->n_routed;
+    a.n_dense_items = (lists->n_routed + kTileQ - 1) / kTileQ;
+    a.win_f = prm->win_f;
+    a.win_h = prm->win_h;
+    a.win_w = prm->win_w;
+    a.n_items = prob->heads * (a.n_dense_items + a.n_qb);
+  } else {
+    return STA_ERR_ARG;
+  }
+  const __nv_bfloat16 *qb, *kb, *vb;
+  st = stage_inputs(prob, q, k, v, workspace, workspace_bytes, &qb, &kb, &vb, s);
+  if (st != STA_OK) return st;
+  return run_attention(prob, a, qb, kb, vb, prm->kv_unit, s);
+}
+
+sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void* k,
+                              const void* v, float scale, void* o, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  sta_status st = check_problem(prob);
+  if (st != STA_OK) return st;
+  if (!q || !k || !v || !o) return STA_ERR_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int N = prob->F * prob->H * prob->W;
+  AttnArgs a = {};
+  a.heads = prob->heads;
+  a.N = N;
+  a.F = prob->F;
+  a.H = prob->H;
+  a.W = prob->W;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf(static_cast<float>(prob->d));
+  a.scale_log2 = sc * 1.4426950408889634f;
+  a.mode = kModeDense;
+  a.block_q = kTileQ;
+  a.n_qb = (N + kTileQ - 1) / kTileQ;
+  a.n_items = prob->heads * a.n_qb;
+  a.o = o;
+  a.out_f32 = prob->dtype == STA_F32;
+  a.dev_status = dev_status;
+  const __nv_bfloat16 *qb, *kb, *vb;
+  st = stage_inputs(prob, q, k, v, workspace, workspace_bytes, &qb, &kb, &vb, s);
+  if (st != STA_OK) return st;
+  return run_attention(prob, a, qb, kb, vb, kTileK, s);
+}
+
+}  // extern "C"
