@@ -7,7 +7,7 @@
 // with s_ik = scale * q_i.k_k; keys outside the listed units never enter the
 // softmax; w_k = 1/pi of the key's sampled unit (stored as -ln pi) or 1.
 //
-// How (one persistent CTA per SM, 6 warps):
+// How (one persistent CTA per SM, 10 warps):
 //   warp 0      producer: TMA loads of the 128-row Q tile and, per 128-key
 //               tile, of the listed key/value units (kv_unit rows each,
 //               128-byte swizzle) into a K ring and a V ring; gathered query
@@ -20,12 +20,14 @@
 //               MN-major in shared memory.  QK of tile t+1 is issued before
 //               PV of tile t, so the tensor core works on the next tile while
 //               the softmax warps handle the current one.
-//   warps 2-5   softmax: thread r owns query row r (TMEM lane r): loads its
-//               128 logits, masks partial units / window, adds log-weights,
-//               keeps a running max and sum in registers (max updates that
-//               move by <= 8 in log2 units are deferred, so O in TMEM is
-//               rescaled only on large jumps), writes P as bf16 into TMEM,
-//               and finally normalises O and stores it.
+//   warps 2-9   softmax, two groups of 4 warps: query row r (TMEM lane r)
+//               is shared by one thread of each group, each taking 64 of the
+//               128 logits of a tile: masks partial units / window, adds
+//               log-weights, keeps a running max (exchanged between the two
+//               halves) and a partial sum in registers (max updates that move
+//               by <= 8 in log2 units are deferred, so O in TMEM is rescaled
+//               only on large jumps), writes P as bf16 into TMEM, and finally
+//               normalises its half of O and stores it.
 // Every wait is bounded; a timeout raises STA_DEV_TIMEOUT, sets a CTA-wide
 // abort flag and unwinds without trapping.
 #include <cuda.h>
@@ -39,10 +41,24 @@
 namespace sta {
 namespace {
 
-constexpr int kThreads = 192;
+// Warp 0 producer, warp 1 MMA issuer, warps 2-9 two softmax groups.
+constexpr int kThreads = 320;
 constexpr int kHalfBytes = 128 * 128;  // 128 rows x 128 bytes: one 64-column half of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+// Tuning constants (compile-time).  One exponential pair in every
+// STA_POLY_EVERY pairs of a full tile goes to the FMA-pipe polynomial
+// (0 = all on MUFU); K/V ring depths.
+#ifndef STA_POLY_EVERY
+#define STA_POLY_EVERY 0
+#endif
+#ifndef STA_KSTAGES
+#define STA_KSTAGES 2
+#endif
+#ifndef STA_VSTAGES
+#define STA_VSTAGES 2
+#endif
 
 template <int D, int KS, int VS>
 struct Layout {
@@ -53,21 +69,25 @@ struct Layout {
   static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
   // barriers: q_full, q_empty, k_full[KS], k_empty[KS], v_full[VS],
-  // v_empty[VS], s_full[2], p_full[2], o_done[2], mma_done
-  static constexpr int NBAR = 2 + 2 * KS + 2 * VS + 7;
-  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  // v_empty[VS], s_full[2], p_full[2], o_done[2], mma_done, then the row
+  // exchange barriers of the two softmax groups: xbar[2][4], lbar[4]
+  static constexpr int NBAR = 2 + 2 * KS + 2 * VS + 7 + 12;
+  static constexpr int OFF_RED = OFF_BAR + NBAR * 8;
+  // red_max[2 parity][2 groups][128 rows], red_l[2 groups][128 rows] (fp32)
+  static constexpr int OFF_MISC = OFF_RED + (2 * 2 * 128 + 2 * 128) * 4;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024
 };
 
 struct Item {
-  int head, kind, q_start, q_len, row, gbase, ntiles, unit, upt;
+  int head, kind, q_start, q_len, row, gbase, ntiles, unit, upt, cnt;
 };
 
 __device__ __forceinline__ Item decode_item(const AttnArgs& a, int it) {
   Item I;
   I.gbase = 0;
   I.row = -1;
+  I.cnt = 0;
   if (a.mode == kModeRouted) {
     const int nd = a.heads * a.n_dense_items;
     if (it < nd) {
@@ -101,6 +121,7 @@ __device__ __forceinline__ Item decode_item(const AttnArgs& a, int it) {
     I.upt = kTileK / a.unit;
     int c = __ldg(a.cnt + I.row);
     c = max(0, min(c, a.cap));
+    I.cnt = c;
     I.ntiles = (c + I.upt - 1) / I.upt;
   }
   return I;
@@ -118,9 +139,7 @@ __device__ __forceinline__ int slot_unit(const AttnArgs& a, const Item& I, int t
     return t;
   }
   const int pos = t * I.upt + s;
-  int c = __ldg(a.cnt + I.row);
-  c = max(0, min(c, a.cap));
-  if (pos >= c) {
+  if (pos >= I.cnt) {
     nvalid = 0;
     return 0;
   }
@@ -170,48 +189,303 @@ __device__ __forceinline__ void load_tile_info(const AttnArgs& a, const Item& I,
   }
 }
 
-// Raw logits of one thread's row -> masked/biased raw logits in place.
-template <int UNIT>
-__device__ __forceinline__ void mask_and_bias(float (&x)[128], const TileInfo<UNIT>& ti,
-                                              bool window, const AttnArgs& a, int fq, int hq,
-                                              int wq) {
-  constexpr int UPT = TileInfo<UNIT>::UPT;
+// Masks (partial units, key tokens past N), log-weights and the local
+// window for the 64 logit columns [WG*64, WG*64+64) one softmax group owns.
+template <int UNIT, int WG>
+__device__ __forceinline__ void mask_half(float (&x)[64], const TileInfo<UNIT>& ti, bool window,
+                                          const AttnArgs& a, int fq, int hq, int wq) {
+  constexpr int CB = WG * 64;
   if (!ti.full) {
 #pragma unroll
-    for (int c = 0; c < 128; ++c) {
-      if ((c % UNIT) >= ti.nv[c / UNIT]) x[c] = -INFINITY;
+    for (int c = 0; c < 64; ++c) {
+      const int cc = CB + c;
+      if ((cc % UNIT) >= ti.nv[cc / UNIT]) x[c] = -INFINITY;
     }
   }
   if (ti.bias) {
 #pragma unroll
-    for (int c = 0; c < 128; ++c) x[c] += ti.braw[c / UNIT];
+    for (int c = 0; c < 64; ++c) x[c] += ti.braw[(CB + c) / UNIT];
   }
   if (window) {
+    // key coordinates advance column by column; they are recomputed from the
+    // unit's first token at every unit boundary (all indices compile-time)
     const int S = a.H * a.W;
+    int f = 0, h = 0, w = 0;
 #pragma unroll
-    for (int s = 0; s < UPT; ++s) {
-      const int t0 = ti.base[s];
-      int f = t0 / S;
-      int rem = t0 - f * S;
-      int h = rem / a.W;
-      int w = rem - h * a.W;
-#pragma unroll
-      for (int e = 0; e < UNIT; ++e) {
-        const int c = s * UNIT + e;
-        const int df = f - fq, dh = h - hq, dw = w - wq;
-        const bool in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
-                        (dh < a.win_h) && (dw >= -a.win_w) && (dw < a.win_w);
-        if (!in) x[c] = -INFINITY;
-        if (++w == a.W) {
-          w = 0;
-          if (++h == a.H) {
-            h = 0;
-            ++f;
-          }
+    for (int c = 0; c < 64; ++c) {
+      const int cc = CB + c;
+      if (c == 0 || (cc % UNIT) == 0) {
+        const int t0 = ti.base[cc / UNIT] + (cc % UNIT);
+        f = t0 / S;
+        const int rem = t0 - f * S;
+        h = rem / a.W;
+        w = rem - h * a.W;
+      }
+      const int df = f - fq, dh = h - hq, dw = w - wq;
+      const bool in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
+                      (dh < a.win_h) && (dw >= -a.win_w) && (dw < a.win_w);
+      if (!in) x[c] = -INFINITY;
+      if (++w == a.W) {
+        w = 0;
+        if (++h == a.H) {
+          h = 0;
+          ++f;
         }
       }
     }
   }
+}
+
+struct SoftmaxShared {
+  uint64_t* s_full;
+  uint64_t* p_full;
+  uint64_t* o_done;
+  uint64_t* xbar;   // [2 parity][4 quadrants], 64 arrivals
+  uint64_t* lbar;   // [4 quadrants], 64 arrivals
+  float* red_max;   // [2 parity][2 groups][128 rows]
+  float* red_l;     // [2 groups][128 rows]
+  volatile int* abort;
+};
+
+__device__ __forceinline__ float nan_flag() { return __int_as_float(0x7fc00000); }
+
+// Softmax warpgroup WG (4 warps).  Thread (quadrant q, lane l) owns query
+// row r = 32q + l of the tile and, of each 128-key tile, the 64 logits
+// [WG*64, WG*64+64); the partner thread of the other group owns the other
+// half of the same row.  Per tile the two exchange their raw row maxima
+// through shared memory (bounded mbarrier, no bar.sync: a partner that gave
+// up cannot block this one), so both apply the same running maximum; each
+// keeps its own partial row sum, combined in the epilogue.  P (bf16) is
+// written over the group's own logit columns; each group rescales and
+// stores its half of O's columns.
+template <int D, int UNIT, int WG>
+__device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxShared& sh,
+                                             uint32_t tmem, int warp, int lane) {
+  constexpr int CB = WG * 64;   // first logit / P column of this group in an S buffer
+  constexpr int OH = D / 2;     // O columns per group
+  constexpr int OB = WG * OH;   // first O column of this group
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;
+  const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+  const float scale_log2 = a.scale_log2;
+  const float inv_scale = kLog2e / scale_log2;  // natural-log weight -> raw logit units
+  const uint64_t limit = kWaitLimitNs;
+  volatile int* abort = sh.abort;
+  uint32_t g = 0, nitem = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
+    if (*abort) break;
+    const Item I = decode_item(a, it);
+    int tok = -1;
+    if (I.kind == kItemGatherDense) {
+      if (r < I.q_len) tok = __ldg(a.routed_ids + I.gbase + r);
+    } else if (r < I.q_len) {
+      tok = I.q_start + r;
+    }
+    bool active = tok >= 0;
+    if (active && I.kind == kItemLocal && __ldg(a.routed_flag + tok)) active = false;
+    const size_t orow = static_cast<size_t>(I.head) * a.N + (tok < 0 ? 0 : tok);
+    if (I.ntiles == 0) {
+      if (active) {
+        if (a.out_f32) {
+          float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D + OB);
+          for (int i = 0; i < OH / 4; ++i) op[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          uint4* op =
+              reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D + OB);
+          for (int i = 0; i < OH / 8; ++i) op[i] = make_uint4(0, 0, 0, 0);
+        }
+        raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
+      }
+      continue;
+    }
+    int fq = 0, hq = 0, wq = 0;
+    const bool window = (I.kind == kItemLocal);
+    if (window && tok >= 0) {
+      const int S = a.H * a.W;
+      fq = tok / S;
+      const int rem = tok - fq * S;
+      hq = rem / a.W;
+      wq = rem - hq * a.W;
+    }
+    const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int t = 0; t < I.ntiles; ++t) {
+      const uint32_t gg = g + t;
+      const uint32_t sb = gg & 1;
+      // Tile metadata first: its global loads overlap the wait for S.
+      TileInfo<kTileK> td;
+      TileInfo<UNIT> ti;
+      bool simple;  // no masked column, no weight, no window
+      if (dense_like) {
+        load_tile_info<kTileK>(a, I, t, inv_scale, td);
+        simple = td.full;
+      } else {
+        load_tile_info<UNIT>(a, I, t, inv_scale, ti);
+        simple = ti.full && !ti.bias && !window;
+      }
+      const bool okw = mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit);
+      float x[64];
+      float mloc = -INFINITY;
+      if (okw) {
+        tc_fence_after();
+        uint32_t v0[32], v1[32];
+        const uint32_t ts = tmem + lane_off + sb * 128 + CB;
+        tmem_ld32(ts, v0);
+        tmem_ld32(ts + 32, v1);
+        tmem_wait_ld();
+        tmem_regs_ready(v0);
+        tmem_regs_ready(v1);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          x[i] = __uint_as_float(v0[i]);
+          x[32 + i] = __uint_as_float(v1[i]);
+        }
+        if (!simple) {
+          if (dense_like)
+            mask_half<kTileK, WG>(x, td, false, a, 0, 0, 0);
+          else
+            mask_half<UNIT, WG>(x, ti, window, a, fq, hq, wq);
+        }
+        float mv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) mv[j] = x[j];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) mv[c & 7] = fmaxf(mv[c & 7], x[c]);
+        mloc = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+                     fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+      }
+      // exchange the row maximum with the partner thread
+      float* rm = sh.red_max + sb * 256;
+      rm[WG * 128 + r] = okw ? mloc : nan_flag();
+      mbar_arrive(sh.xbar + sb * 4 + quad);
+      const bool okx = mbar_wait(sh.xbar + sb * 4 + quad, (gg >> 1) & 1, abort, limit);
+      const float mo = rm[(1 - WG) * 128 + r];
+      if (!okw || !okx || mo != mo) {
+        ok = false;
+        break;
+      }
+      const float m_tile = fmaxf(mloc, mo) * scale_log2;  // -inf if all masked
+      const float m_new = fmaxf(m_run, m_tile);
+      const bool need = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
+      if (__any_sync(0xffffffffu, need)) {
+        // O rows of this warp hold tiles < t; the last of them must be
+        // accumulated before it is rescaled.
+        const uint32_t gp = gg - 1;
+        if (!mbar_wait(sh.o_done + (gp & 1), (gp >> 1) & 1, abort, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = need ? fast_exp2(m_run - m_new) : 1.f;
+#pragma unroll
+        for (int ch = 0; ch < OH / 32; ++ch) {
+          uint32_t v[32];
+          const uint32_t to = tmem + lane_off + 256 + OB + ch * 32;
+          tmem_ld32(to, v);
+          tmem_wait_ld();
+          tmem_regs_ready(v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+          tmem_st32(to, v);
+        }
+        tmem_wait_st();
+        if (need) {
+          l_run *= f;
+          m_run = m_new;
+        }
+      }
+      if (m_run == -INFINITY) m_run = m_new;
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      float ls[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ls[j] = 0.f;
+      uint32_t pk[32];
+      if (simple) {
+        // part of the exponentials on the FMA pipe, the rest on MUFU
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float a0 = fmaf(x[c], scale_log2, -m_use);
+          const float a1 = fmaf(x[c + 1], scale_log2, -m_use);
+          float p0, p1;
+          if (STA_POLY_EVERY > 0 && ((c >> 1) % (STA_POLY_EVERY > 0 ? STA_POLY_EVERY : 1)) ==
+                                        (STA_POLY_EVERY > 0 ? STA_POLY_EVERY - 1 : 0)) {
+            p0 = exp2_poly(a0);
+            p1 = exp2_poly(a1);
+          } else {
+            p0 = fast_exp2(a0);
+            p1 = fast_exp2(a1);
+          }
+          ls[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float p0 = fast_exp2(fmaf(x[c], scale_log2, -m_use));
+          const float p1 = fast_exp2(fmaf(x[c + 1], scale_log2, -m_use));
+          ls[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = pack_bf16x2(p0, p1);
+        }
+      }
+      l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+      tmem_st32(tmem + lane_off + sb * 128 + CB, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(sh.p_full + sb);
+    }
+    if (!ok) break;
+    // ------------------------------------------------------------ epilogue
+    const uint32_t gl = g + I.ntiles - 1;
+    const bool okw = mbar_wait(sh.o_done + (gl & 1), (gl >> 1) & 1, abort, limit);
+    g += I.ntiles;
+    sh.red_l[WG * 128 + r] = okw ? l_run : nan_flag();
+    mbar_arrive(sh.lbar + quad);
+    const bool okx = mbar_wait(sh.lbar + quad, nitem & 1, abort, limit);
+    ++nitem;
+    const float lo = sh.red_l[(1 - WG) * 128 + r];
+    if (!okw || !okx || lo != lo) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    const float l_tot = l_run + lo;
+    const bool empty = !(l_tot > 0.f);
+    const float inv_l = empty ? 0.f : 1.f / l_tot;
+    if (WG == 0 && active && empty) raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
+#pragma unroll
+    for (int ch = 0; ch < OH / 32; ++ch) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + 256 + OB + ch * 32, v);
+      tmem_wait_ld();
+      tmem_regs_ready(v);
+      if (active) {
+        const size_t col = orow * D + OB + ch * 32;
+        if (a.out_f32) {
+          float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.o) + col);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            op[i] = make_float4(
+                __uint_as_float(v[4 * i]) * inv_l, __uint_as_float(v[4 * i + 1]) * inv_l,
+                __uint_as_float(v[4 * i + 2]) * inv_l, __uint_as_float(v[4 * i + 3]) * inv_l);
+        } else {
+          uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + col);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            op[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]) * inv_l,
+                                           __uint_as_float(v[8 * i + 1]) * inv_l),
+                               pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l,
+                                           __uint_as_float(v[8 * i + 3]) * inv_l),
+                               pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l,
+                                           __uint_as_float(v[8 * i + 5]) * inv_l),
+                               pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l,
+                                           __uint_as_float(v[8 * i + 7]) * inv_l));
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  if (!ok) fail(abort, a.dev_status);
 }
 
 template <int D, int KS, int VS, int UNIT>
@@ -240,6 +514,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* mma_done = o_done + 2;
+  uint64_t* xbar = mma_done + 1;  // [2][4]
+  uint64_t* lbar = xbar + 8;      // [4]
+  float* red_max = reinterpret_cast<float*>(smem + L::OFF_RED);
+  float* red_l = red_max + 2 * 2 * 128;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -259,10 +537,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 128);
+      mbar_init(p_full + i, 256);
       mbar_init(o_done + i, 1);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(xbar + i, 64);
+    for (int i = 0; i < 4; ++i) mbar_init(lbar + i, 64);
     *abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
@@ -400,7 +680,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
           const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024);
-          mma_bf16_ts(tO, tS + kk * 8, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          // P of keys 0..63 sits in columns 0..31 of the S buffer, keys
+          // 64..127 in columns 64..95 (each softmax group writes over its
+          // own logits)
+          const uint32_t pa = tS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+          mma_bf16_ts(tO, pa, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
         }
         mma_commit(v_empty + st);
         ++vt;
@@ -458,179 +742,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const float scale_log2 = a.scale_log2;
-    const float inv_scale = kLog2e / scale_log2;  // natural-log weight -> raw logit units
-    uint32_t g = 0;
-    bool ok = true;
-    for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
-      if (*abort) break;
-      const Item I = decode_item(a, it);
-      int tok = -1;
-      if (I.kind == kItemGatherDense) {
-        if (r < I.q_len) tok = __ldg(a.routed_ids + I.gbase + r);
-      } else if (r < I.q_len) {
-        tok = I.q_start + r;
-      }
-      bool active = tok >= 0;
-      if (active && I.kind == kItemLocal && __ldg(a.routed_flag + tok)) active = false;
-      const size_t orow = static_cast<size_t>(I.head) * a.N + (tok < 0 ? 0 : tok);
-      if (I.ntiles == 0) {
-        if (active) {
-          if (a.out_f32) {
-            float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D);
-            for (int i = 0; i < D / 4; ++i) op[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          } else {
-            uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D);
-            for (int i = 0; i < D / 8; ++i) op[i] = make_uint4(0, 0, 0, 0);
-          }
-          raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
-        }
-        continue;
-      }
-      int fq = 0, hq = 0, wq = 0;
-      const bool window = (I.kind == kItemLocal);
-      if (window && tok >= 0) {
-        const int S = a.H * a.W;
-        fq = tok / S;
-        const int rem = tok - fq * S;
-        hq = rem / a.W;
-        wq = rem - hq * a.W;
-      }
-      const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
-      float m_run = -INFINITY, l_run = 0.f;
-      for (int t = 0; t < I.ntiles; ++t) {
-        const uint32_t gg = g + t;
-        const uint32_t sb = gg & 1;
-        if (!mbar_wait(s_full + sb, (gg >> 1) & 1, abort, limit)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        float x[128];
-        {
-          uint32_t v[32];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            tmem_ld32(tmem + lane_off + sb * 128 + j * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[j * 32 + i] = __uint_as_float(v[i]);
-          }
-        }
-        if (dense_like) {
-          TileInfo<kTileK> ti;
-          load_tile_info<kTileK>(a, I, t, inv_scale, ti);
-          mask_and_bias<kTileK>(x, ti, false, a, 0, 0, 0);
-        } else {
-          TileInfo<UNIT> ti;
-          load_tile_info<UNIT>(a, I, t, inv_scale, ti);
-          mask_and_bias<UNIT>(x, ti, window, a, fq, hq, wq);
-        }
-        float mx = x[0];
-#pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
-        const float m_tile = mx * scale_log2;  // -inf if all masked
-        const float m_new = fmaxf(m_run, m_tile);
-        const bool need = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
-        if (__any_sync(0xffffffffu, need)) {
-          // O of this warp's rows holds tiles < t; the last of them must be
-          // accumulated before it is rescaled.
-          const uint32_t gp = gg - 1;
-          if (!mbar_wait(o_done + (gp & 1), (gp >> 1) & 1, abort, limit)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float f = need ? fast_exp2(m_run - m_new) : 1.f;
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_off + 256 + ch * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-            tmem_st32(tmem + lane_off + 256 + ch * 32, v);
-          }
-          tmem_wait_st();
-          if (need) {
-            l_run *= f;
-            m_run = m_new;
-          }
-        }
-        if (m_run == -INFINITY) m_run = m_new;
-        const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-        float lsum = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = fast_exp2(fmaf(x[c], scale_log2, -m_use));
-          const float p1 = fast_exp2(fmaf(x[c + 1], scale_log2, -m_use));
-          lsum += p0 + p1;
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-        }
-        l_run += lsum;
-        {
-          uint32_t v[32];
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = pk[j * 32 + i];
-            tmem_st32(tmem + lane_off + sb * 128 + j * 32, v);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full + sb);
-      }
-      if (!ok) break;
-      // ---------------------------------------------------------- epilogue
-      const uint32_t gl = g + I.ntiles - 1;
-      if (!mbar_wait(o_done + (gl & 1), (gl >> 1) & 1, abort, limit)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      g += I.ntiles;
-      const bool empty = !(l_run > 0.f);
-      const float inv_l = empty ? 0.f : 1.f / l_run;
-      if (active && empty) raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + 256 + ch * 32, v);
-        tmem_wait_ld();
-        if (active) {
-          if (a.out_f32) {
-            float4* op =
-                reinterpret_cast<float4*>(static_cast<float*>(a.o) + orow * D + ch * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              op[i] = make_float4(__uint_as_float(v[4 * i]) * inv_l,
-                                  __uint_as_float(v[4 * i + 1]) * inv_l,
-                                  __uint_as_float(v[4 * i + 2]) * inv_l,
-                                  __uint_as_float(v[4 * i + 3]) * inv_l);
-          } else {
-            uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + orow * D +
-                                                 ch * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              op[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]) * inv_l,
-                                             __uint_as_float(v[8 * i + 1]) * inv_l),
-                                 pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l,
-                                             __uint_as_float(v[8 * i + 3]) * inv_l),
-                                 pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l,
-                                             __uint_as_float(v[8 * i + 5]) * inv_l),
-                                 pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l,
-                                             __uint_as_float(v[8 * i + 7]) * inv_l));
-          }
-        }
-      }
-      tc_fence_before();
-    }
-    if (!ok) fail(abort, a.dev_status);
+    SoftmaxShared sh{s_full, p_full, o_done, xbar, lbar, red_max, red_l, abort};
+    if (warp < 6)
+      softmax_role<D, UNIT, 0>(a, sh, tmem, warp, lane);
+    else
+      softmax_role<D, UNIT, 1>(a, sh, tmem, warp, lane);
   }
 
   tc_fence_before();
@@ -670,7 +786,7 @@ cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tq,
                              cudaStream_t stream) {
 #define STA_ATTN_CASE(DD, UU)                                                                \
   if (d == DD && a.unit == UU)                                                               \
-    return launch_t<DD, 2, 2, UU>(a, tq, tku, tvu, tkf, tvf, num_sms, stream);
+    return launch_t<DD, STA_KSTAGES, STA_VSTAGES, UU>(a, tq, tku, tvu, tkf, tvf, num_sms, stream);
   STA_ATTN_CASE(128, 128)
   STA_ATTN_CASE(128, 64)
   STA_ATTN_CASE(128, 32)

@@ -173,6 +173,21 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+
+// Ties the registers of an earlier tcgen05.ld to a point after
+// tmem_wait_ld(): every later use depends on this (ordered) statement, so the
+// compiler cannot move a read of the registers above the wait.
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -213,6 +228,24 @@ __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA/ALU pipes, for finite x >= -125 (the caller clamps; masked
+// -inf entries never take this path).  x = j + f with j = nearest integer
+// (obtained by adding 1.5*2^23, which leaves j in the low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f is a cubic fitted by the Remez exchange algorithm on
+// relative error (coefficients from csrc/fit_exp2_poly.py; max relative
+// error 7.5e-5, far below the bf16 rounding of P); 2^j is added to the
+// exponent field: (bits(x + 1.5*2^23) << 23) == j << 23 modulo 2^32.
+__device__ __forceinline__ float exp2_poly(float x) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.999928057f, c1 = 0.693260968f, c2 = 0.242611125f, c3 = 0.0551716685f;
+  x = fmaxf(x, -125.0f);
+  const float t = __fadd_rn(x, kShift);
+  const float j = __fsub_rn(t, kShift);
+  const float f = __fsub_rn(x, j);
+  const float p = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, c0);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 }  // namespace sta
