@@ -1,6 +1,6 @@
 """Build libsta.so in-tree with nvcc for sm_100a.
 
-    python -m sparse_spatiotemporal_attention_video_b200.build [--verbose]
+    python sparse_spatiotemporal_attention_video_b200/build.py [--verbose]
 
 Every .cu file under csrc/ is compiled to an object (in parallel), then
 linked into one shared library next to this file.  No torch types cross the
