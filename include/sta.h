@@ -18,7 +18,8 @@
  * - Every pointer argument that names tensor data is a DEVICE pointer owned
  *   by the caller.  The library never allocates, frees or retains memory and
  *   keeps no state between calls.  Scratch space, where needed, is passed in
- *   as `workspace` after querying its size.
+ *   as `workspace` after querying its size.  (The one exception is
+ *   sta_sparse_attn_fwd_noalloc, which uses a fixed array of its own.)
  * - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
  *   legacy default stream) and returns.  Results are valid once the caller
  *   has synchronised the stream.
@@ -216,6 +217,32 @@ sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void
                               const void* v, float scale, void* o,
                               void* workspace, size_t workspace_bytes,
                               int32_t* dev_status, sta_stream_t stream);
+
+/*
+ * sta_sparse_attn_fwd with no workspace argument, for callers that cannot
+ * allocate device memory: a plugin that its host framework hands only the
+ * input and output buffers, or a pipeline that bans cudaMalloc after
+ * start-up because it can synchronise the device.  (The pages have no
+ * counterpart: this is a deployment convenience of this library.)
+ *
+ * Same arguments and results as sta_sparse_attn_fwd.  bf16 inputs need no
+ * scratch.  fp32 inputs are rounded to bf16 into one fixed 12 MiB device
+ * array inside the library (never cudaMalloc), so 3 * heads*N*d bf16
+ * copies, each rounded up to 256 bytes, must fit in 12 MiB: at most
+ * 2,097,152 elements per tensor; larger problems return STA_ERR_WORKSPACE
+ * and enqueue nothing.  Each device the library is used on holds the array
+ * until the process exits.
+ * The first call on a device looks the array's device address up (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  Every call on every stream shares the one array and leaves its
+ * contents behind: two fp32 calls that may overlap on the GPU (different
+ * streams, no ordering between them) race on it.  Calls on one stream are
+ * ordered and safe.
+ */
+sta_status sta_sparse_attn_fwd_noalloc(const sta_problem* prob, const sta_attn_params* prm,
+                                       const void* q, const void* k, const void* v,
+                                       const sta_block_lists* lists, void* o,
+                                       int32_t* dev_status, sta_stream_t stream);
 
 /* Static description of a status code / of the device status bits. */
 const char* sta_status_string(sta_status s);

@@ -74,6 +74,11 @@ SIGNATURES = {
                                            ctypes.POINTER(BlockLists), ctypes.c_void_p,
                                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
                                            ctypes.c_void_p]),
+    "sta_sparse_attn_fwd_noalloc": (ctypes.c_int, [ctypes.POINTER(Problem),
+                                                   ctypes.POINTER(AttnParams), ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_void_p,
+                                                   ctypes.POINTER(BlockLists), ctypes.c_void_p,
+                                                   ctypes.c_void_p, ctypes.c_void_p]),
     "sta_dense_attn_fwd": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p,
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
@@ -94,7 +99,7 @@ def load(path=LIB_PATH):
     if not os.path.exists(path):
         raise ImportError(
             f"{path} is missing: build it with "
-            "`python -m sparse_spatiotemporal_attention_video_b200.build` (nvcc, sm_100a)")
+            "`python sparse_spatiotemporal_attention_video_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

@@ -67,6 +67,17 @@ def sta_sparse_attn_fwd(prob, prm: AttnParams, q, k, v, lists: BlockLists, o, wo
           "sta_sparse_attn_fwd")
 
 
+def sta_sparse_attn_fwd_noalloc(prob, prm: AttnParams, q, k, v, lists: BlockLists, o,
+                                dev_status=None, stream=None):
+    """sta_sparse_attn_fwd without a workspace: fp32 inputs are staged in
+    the library's fixed device array (see include/sta.h)."""
+    lib = _lib.load()
+    check(lib.sta_sparse_attn_fwd_noalloc(ctypes.byref(prob), ctypes.byref(prm), _ptr(q),
+                                          _ptr(k), _ptr(v), ctypes.byref(lists), _ptr(o),
+                                          _ptr(dev_status), _stream(stream)),
+          "sta_sparse_attn_fwd_noalloc")
+
+
 def sta_dense_attn_fwd(prob, q, k, v, scale, o, workspace=None, workspace_bytes=0,
                        dev_status=None, stream=None):
     lib = _lib.load()

@@ -289,3 +289,70 @@ sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// sta_sparse_attn_fwd_noalloc: sparse attention for callers that cannot
+// allocate device memory.
+//
+// The only scratch the attention path needs is the bf16 copy of fp32 q, k, v
+// that the tensor cores read.  sta_sparse_attn_fwd takes it from a caller
+// workspace; this variant takes it from the fixed array below instead.  It
+// is for callers that cannot allocate: a plugin that its host framework hands
+// only the input and output buffers, with no access to the framework's
+// allocator, or a latency-bound pipeline that bans allocation after start-up
+// because cudaMalloc can synchronise the device and stall other streams.
+//
+// The array is part of the library's device image: each device the library
+// is used on holds kStaticStageBytes until the process exits.  Host code
+// cannot use the symbol's name as a device address (it names a host-side
+// shadow), so its device address is looked up once per device with
+// cudaGetSymbolAddress and cached.
+namespace {
+
+constexpr size_t kStaticStageBytes = size_t(12) << 20;  // 12 MiB
+constexpr int kMaxStaticDevices = 64;
+
+static __device__ __align__(256) uint8_t g_static_stage[kStaticStageBytes];
+
+std::mutex g_static_stage_mu;
+void* g_static_stage_ptr[kMaxStaticDevices] = {};
+
+// Device address of g_static_stage on the current device (set-up on the
+// first call per device).
+sta_status static_stage_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return STA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxStaticDevices) return STA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_stage_mu);
+  if (!g_static_stage_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_stage) != cudaSuccess || !p) return STA_ERR_CUDA;
+    g_static_stage_ptr[dev] = p;
+  }
+  *out = g_static_stage_ptr[dev];
+  return STA_OK;
+}
+
+}  // namespace
+
+extern "C" sta_status sta_sparse_attn_fwd_noalloc(const sta_problem* prob,
+                                                  const sta_attn_params* prm, const void* q,
+                                                  const void* k, const void* v,
+                                                  const sta_block_lists* lists, void* o,
+                                                  int32_t* dev_status, sta_stream_t stream) {
+  sta_status st = check_problem(prob);
+  if (st != STA_OK) return st;
+  if (prob->dtype != STA_F32) {
+    // bf16 inputs feed the tensor cores directly: no scratch at all.
+    return sta_sparse_attn_fwd(prob, prm, q, k, v, lists, o, nullptr, 0, dev_status, stream);
+  }
+  const size_t need = 3 * staged_bytes(prob);
+  if (need > kStaticStageBytes) return STA_ERR_WORKSPACE;
+  void* stage = nullptr;
+  st = static_stage_address(&stage);
+  if (st != STA_OK) return st;
+  // Every byte the kernels read from the stage is written by this call's
+  // conversion first, so nothing needs clearing.
+  return sta_sparse_attn_fwd(prob, prm, q, k, v, lists, o, stage, kStaticStageBytes, dev_status,
+                             stream);
+}
