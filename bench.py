@@ -36,7 +36,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of attn_fwd.cu, first 16 hex).
-NCU_TRAFFIC = {"source_sha": None, "bytes_per_launch": None}
+NCU_TRAFFIC = {"source_sha": "61bd247adb317a0a", "bytes_per_launch": 303713280 + 87362304}
 
 
 def parse():
