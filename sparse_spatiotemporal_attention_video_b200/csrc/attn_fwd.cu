@@ -27,7 +27,12 @@
 //               halves) and a partial sum in registers (max updates that move
 //               by <= 8 in log2 units are deferred, so O in TMEM is rescaled
 //               only on large jumps), writes P as bf16 into TMEM, and finally
-//               normalises its half of O and stores it.
+//               normalises its half of O and stores it.  The row sum adds the
+//               bf16-rounded P the tensor core multiplies, not the fp32
+//               values: numerator and denominator then carry the same
+//               weights, so a dominant key's rounding error scales with
+//               (v - O) instead of v (with a deferred maximum its weight is
+//               not exactly 1, and summing fp32 P doubled the output error).
 // Every wait is bounded; a timeout raises STA_DEV_TIMEOUT, sets a CTA-wide
 // abort flag and unwinds without trapping.
 #include <cuda.h>
@@ -45,7 +50,6 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kHalfBytes = 128 * 128;  // 128 rows x 128 bytes: one 64-column half of a tile
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 // Tuning constants (compile-time).  One exponential pair in every
 // STA_POLY_EVERY pairs of a full tile goes to the FMA-pipe polynomial
@@ -53,6 +57,12 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 #ifndef STA_POLY_EVERY
 #define STA_POLY_EVERY 0
 #endif
+// Deferred rescale: the running row maximum moves (and O is rescaled) only
+// when a tile's maximum exceeds it by more than this many log2 units.
+#ifndef STA_RESCALE_THRESHOLD
+#define STA_RESCALE_THRESHOLD 8.0f
+#endif
+constexpr float kRescaleThreshold = STA_RESCALE_THRESHOLD;
 #ifndef STA_KSTAGES
 #define STA_KSTAGES 2
 #endif
@@ -416,16 +426,16 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
             p0 = fast_exp2(a0);
             p1 = fast_exp2(a1);
           }
-          ls[(c >> 1) & 7] += p0 + p1;
           pk[c >> 1] = pack_bf16x2(p0, p1);
+          ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
         }
       } else {
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           const float p0 = fast_exp2(fmaf(x[c], scale_log2, -m_use));
           const float p1 = fast_exp2(fmaf(x[c + 1], scale_log2, -m_use));
-          ls[(c >> 1) & 7] += p0 + p1;
           pk[c >> 1] = pack_bf16x2(p0, p1);
+          ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
         }
       }
       l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));

@@ -69,4 +69,33 @@ cudaError_t launch_radial_lists(int F, int H, int W, int B, int w0, int w_off, i
                                 int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
                                 int32_t* dev_status, cudaStream_t stream);
 
+// Block means (sel_pool.cu): out_i[h][b][d] = mean of the rows of block b of
+// x_i (fp32); x1/out1 may be null.
+cudaError_t launch_block_means(const __nv_bfloat16* x0, const __nv_bfloat16* x1, float* out0,
+                               float* out1, int heads, int N, int d, int U, cudaStream_t s);
+
+// Entropy-radius selector (sel_entropy.cu).
+int entropy_max_blocks(int d);
+cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, int heads, int F, int H,
+                                 int W, int d, int B, float scale, float alpha, float beta,
+                                 int r_lo, int r_hi, int tile_h, int tile_w, int32_t* idx,
+                                 int32_t* cnt, int cap, int32_t* required_cap, float* entropy,
+                                 int32_t* radius, int32_t* dev_status, cudaStream_t s);
+
+// Difficulty routing (sel_routed.cu).
+cudaError_t launch_routed_select(const float* difficulty, int N, int n_routed,
+                                 int32_t* routed_ids, uint8_t* routed_flag, cudaStream_t s);
+cudaError_t launch_routed_local_lists(int F, int H, int W, int B, int U, int win_f, int win_h,
+                                      int win_w, int32_t* idx, int32_t* cnt, int cap,
+                                      int32_t* required_cap, int32_t* dev_status,
+                                      cudaStream_t s);
+
+// Clustering importance + inclusion-probability sampling (sel_ibcs.cu).
+int ibcs_max_subblocks();
+cudaError_t launch_ibcs_sip(const __nv_bfloat16* q, const float* kbar, float* cent, float* wts,
+                            float* p, int heads, int N, int d, int B, int U, int km_k, int iters,
+                            int m, uint64_t seed, float scale, int32_t* idx, float* logw,
+                            int32_t* cnt, int cap, int32_t* required_cap, int32_t* dev_status,
+                            cudaStream_t s);
+
 }  // namespace sta

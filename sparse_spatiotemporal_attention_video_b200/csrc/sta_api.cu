@@ -124,6 +124,48 @@ sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16*
   return STA_OK;
 }
 
+// Workspace carve-up of the content selectors (256-byte aligned segments).
+struct SelWorkspace {
+  size_t qbar = 0, kbar = 0, cent = 0, wts = 0, p = 0, total = 0;
+};
+
+SelWorkspace sel_workspace(const sta_problem* p, const sta_selector_params* sel) {
+  SelWorkspace w;
+  const size_t h = static_cast<size_t>(p->heads);
+  const size_t N = static_cast<size_t>(p->F) * p->H * p->W;
+  const size_t d = static_cast<size_t>(p->d);
+  if (sel->block_q < 1 || sel->kv_unit < 1) return w;
+  const size_t nqb = (N + sel->block_q - 1) / sel->block_q;
+  const size_t nku = (N + sel->kv_unit - 1) / sel->kv_unit;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += round_up(bytes, 256);
+    return at;
+  };
+  if (sel->kind == STA_SEL_ENTROPY) {
+    w.qbar = take(h * nqb * d * 4);
+    w.kbar = take(h * nku * d * 4);
+  } else if (sel->kind == STA_SEL_IBCS_SIP) {
+    const size_t km = sel->km_k > 0 ? static_cast<size_t>(sel->km_k) : 1;
+    w.kbar = take(h * nku * d * 4);
+    w.cent = take(h * nqb * km * d * 4);
+    w.wts = take(h * nqb * km * 4);
+    w.p = take(h * nqb * nku * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+// ceil(frac * n) with a relative slack of 1e-6 (so that a decimal fraction
+// stored in binary does not add one), clamped to [lo, n].
+int fraction_count(double frac, long long n, int lo) {
+  long long m = static_cast<long long>(ceil(frac * static_cast<double>(n) * (1.0 - 1e-6)));
+  if (m < lo) m = lo;
+  if (m > n) m = n;
+  return static_cast<int>(m);
+}
+
 }  // namespace
 
 extern "C" {
@@ -168,16 +210,13 @@ int sta_build_blocks_rows(const sta_problem* prob, const sta_selector_params* se
 
 size_t sta_build_blocks_workspace(const sta_problem* prob, const sta_selector_params* sel) {
   if (check_problem(prob) != STA_OK || !sel) return 0;
-  return 0;
+  const SelWorkspace w = sel_workspace(prob, sel);
+  return w.total;
 }
 
 sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* sel,
                             const void* q, const void* k, sta_block_lists* out, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
-  (void)q;
-  (void)k;
-  (void)workspace;
-  (void)workspace_bytes;
   sta_status st = check_problem(prob);
   if (st != STA_OK) return st;
   if (!sel || !out || !out->idx || !out->cnt || out->cap < 1) return STA_ERR_ARG;
@@ -192,6 +231,79 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       if (launch_radial_lists(prob->F, prob->H, prob->W, sel->block_q, sel->radial_w0,
                               sel->radial_w_off, sel->radial_full_df, out->idx, out->cnt, out->cap,
                               out->required_cap, dev_status, s) != cudaSuccess)
+        return STA_ERR_CUDA;
+      return STA_OK;
+    }
+    case STA_SEL_ENTROPY: {
+      if (prob->dtype != STA_BF16 || !q || !k) return q && k ? STA_ERR_UNSUPPORTED : STA_ERR_ARG;
+      if (sel->kv_unit != sel->block_q) return STA_ERR_UNSUPPORTED;
+      if (sel->ent_r_lo > sel->ent_r_hi || sel->ent_tile_h < 1 || sel->ent_tile_w < 1)
+        return STA_ERR_ARG;
+      const int N = prob->F * prob->H * prob->W;
+      const int nb = (N + sel->block_q - 1) / sel->block_q;
+      if (nb > entropy_max_blocks(prob->d)) return STA_ERR_UNSUPPORTED;
+      const SelWorkspace w = sel_workspace(prob, sel);
+      if (!workspace || workspace_bytes < w.total) return STA_ERR_WORKSPACE;
+      uint8_t* ws = static_cast<uint8_t*>(workspace);
+      float* qbar = reinterpret_cast<float*>(ws + w.qbar);
+      float* kbar = reinterpret_cast<float*>(ws + w.kbar);
+      out->head_shared = 0;
+      const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
+      if (launch_block_means(static_cast<const __nv_bfloat16*>(q),
+                             static_cast<const __nv_bfloat16*>(k), qbar, kbar, prob->heads, N,
+                             prob->d, sel->block_q, s) != cudaSuccess)
+        return STA_ERR_CUDA;
+      if (launch_entropy_lists(qbar, kbar, prob->heads, prob->F, prob->H, prob->W, prob->d,
+                               sel->block_q, scale, sel->ent_alpha, sel->ent_beta, sel->ent_r_lo,
+                               sel->ent_r_hi, sel->ent_tile_h, sel->ent_tile_w, out->idx,
+                               out->cnt, out->cap, out->required_cap, out->entropy, out->radius,
+                               dev_status, s) != cudaSuccess)
+        return STA_ERR_CUDA;
+      return STA_OK;
+    }
+    case STA_SEL_ROUTED: {
+      if (!sel->difficulty || !out->routed_ids || !out->routed_flag) return STA_ERR_ARG;
+      if (sel->win_f < 0 || sel->win_h < 1 || sel->win_w < 1) return STA_ERR_ARG;
+      if (!(sel->dense_frac >= 0.f && sel->dense_frac <= 1.f)) return STA_ERR_ARG;
+      const int N = prob->F * prob->H * prob->W;
+      const int n_routed = fraction_count(sel->dense_frac, N, 0);
+      out->head_shared = 1;
+      out->n_routed = n_routed;
+      if (launch_routed_select(sel->difficulty, N, n_routed, out->routed_ids, out->routed_flag,
+                               s) != cudaSuccess)
+        return STA_ERR_CUDA;
+      if (launch_routed_local_lists(prob->F, prob->H, prob->W, sel->block_q, sel->kv_unit,
+                                    sel->win_f, sel->win_h, sel->win_w, out->idx, out->cnt,
+                                    out->cap, out->required_cap, dev_status, s) != cudaSuccess)
+        return STA_ERR_CUDA;
+      return STA_OK;
+    }
+    case STA_SEL_IBCS_SIP: {
+      if (prob->dtype != STA_BF16 || !q || !k) return q && k ? STA_ERR_UNSUPPORTED : STA_ERR_ARG;
+      if (sel->km_k != 1 && sel->km_k != 2 && sel->km_k != 4 && sel->km_k != 8)
+        return STA_ERR_UNSUPPORTED;
+      if (sel->km_iters < 1) return STA_ERR_ARG;
+      if (!(sel->sample_frac > 0.f && sel->sample_frac <= 1.f)) return STA_ERR_ARG;
+      const int N = prob->F * prob->H * prob->W;
+      const int n_sub = (N + sel->kv_unit - 1) / sel->kv_unit;
+      if (n_sub > ibcs_max_subblocks()) return STA_ERR_UNSUPPORTED;
+      const SelWorkspace w = sel_workspace(prob, sel);
+      if (!workspace || workspace_bytes < w.total) return STA_ERR_WORKSPACE;
+      uint8_t* ws = static_cast<uint8_t*>(workspace);
+      float* kbar = reinterpret_cast<float*>(ws + w.kbar);
+      float* cent = reinterpret_cast<float*>(ws + w.cent);
+      float* wts = reinterpret_cast<float*>(ws + w.wts);
+      float* pbuf = reinterpret_cast<float*>(ws + w.p);
+      out->head_shared = 0;
+      const int m = fraction_count(sel->sample_frac, n_sub, 1);
+      const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
+      if (launch_block_means(static_cast<const __nv_bfloat16*>(k), nullptr, kbar, nullptr,
+                             prob->heads, N, prob->d, sel->kv_unit, s) != cudaSuccess)
+        return STA_ERR_CUDA;
+      if (launch_ibcs_sip(static_cast<const __nv_bfloat16*>(q), kbar, cent, wts, pbuf,
+                          prob->heads, N, prob->d, sel->block_q, sel->kv_unit, sel->km_k,
+                          sel->km_iters, m, sel->seed, scale, out->idx, out->logw, out->cnt,
+                          out->cap, out->required_cap, dev_status, s) != cudaSuccess)
         return STA_ERR_CUDA;
       return STA_OK;
     }

@@ -44,6 +44,41 @@ def selector(w, difficulty=None):
     return s
 
 
+def selector_workspace(w, device="cuda"):
+    """Device scratch of sta_build_blocks for this workload (None if none)."""
+    n = api.sta_build_blocks_workspace(problem(w), selector(w))
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def route_count(w):
+    """Tokens on the dense path: ceil(frac * N) with the library's 1e-6 slack."""
+    N = w["F"] * w["H"] * w["W"]
+    m = math.ceil(float(torch.tensor(w["routed"]["dense_frac"], dtype=torch.float32)) * N
+                  * (1.0 - 1e-6))
+    return max(0, min(N, m))
+
+
+def retained_pairs_routed(w, routed_flag):
+    """Algorithmic kept (query, key) pairs of the routed workload over all
+    heads: N keys for every routed token plus, for every other token, the
+    number of keys inside its clipped local window.  routed_flag: [N] bool
+    or uint8 (host or device)."""
+    F, H, W = w["F"], w["H"], w["W"]
+    N = F * H * W
+    c = w["routed"]
+    flag = routed_flag.detach().cpu().bool()
+    t = torch.arange(N, dtype=torch.int64)
+    S = H * W
+    f, h, x = t // S, (t % S) // W, t % W
+    nf = torch.clamp(f + c["win_f"], max=F - 1) - torch.clamp(f - c["win_f"], min=0) + 1
+    nh = torch.clamp(h + c["win_h"], max=H) - torch.clamp(h - c["win_h"], min=0)
+    nw = torch.clamp(x + c["win_w"], max=W) - torch.clamp(x - c["win_w"], min=0)
+    local = int((nf * nh * nw)[~flag].sum().item())
+    return w["heads"] * (int(flag.sum().item()) * N + local)
+
+
 def attn_params(w):
     p = AttnParams()
     p.mode = STA_ATTN_ROUTED if w["selector"] == "routed" else STA_ATTN_LISTS

@@ -48,7 +48,8 @@ WORKLOADS = {
         heads=12, F=21, H=30, W=52, d=128, dtype="bf16", noise=None,
         noise_block=(0.2, 2.0), logit_std=3.0, block_q=128, kv_unit=128,
         selector="entropy",
-        entropy=dict(alpha=None, beta=None, r_lo=1, r_hi=2, tile_h=8, tile_w=16),
+        entropy=dict(alpha=-208.83056640625, beta=38.206417083740234, r_lo=1, r_hi=2,
+                     tile_h=8, tile_w=16),
         seed=0),
     # HetA-style routing at the Wan2.2-5B shape 31x44x80 (N=109120), 24 heads.
     # Top 20% of tokens by a Beta(2,5) difficulty go to dense attention; the

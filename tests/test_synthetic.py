@@ -29,3 +29,15 @@ def test_region_noise_and_difficulty():
     assert q.shape == (1, 256, 128)
     d = make_difficulty(workload("heta_routed", F=2, H=4, W=8))
     assert d.dtype == np.float32 and d.shape == (64,) and 0 < d.min() and d.max() < 1
+
+
+def test_entropy_workload_uses_the_stored_calibration():
+    import json
+    import os
+    from synthetic import workload
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                        "entropy_calibration.json")
+    cal = json.load(open(path))
+    e = workload("tra_entropy")["entropy"]
+    assert (e["alpha"], e["beta"], e["r_lo"], e["r_hi"]) == (cal["alpha"], cal["beta"],
+                                                             cal["r_lo"], cal["r_hi"])
