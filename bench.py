@@ -1,19 +1,28 @@
-"""Benchmark: radial sparse attention at the Wan2.1-1.3B shape on B200.
+"""Benchmark: one step of the sparse-attention hot path on B200.
 
-One step = the whole hot path on one batch: the radial selector
-(sta_build_blocks) and the block-sparse attention (sta_sparse_attn_fwd) over
-12 heads x 32760 tokens x d=128, bf16.  Reported:
+Default workload: static radial sparse attention at the Wan2.1-1.3B latent
+grid (12 heads x 21x30x52 = 32,760 tokens x d=128, bf16, 128-token blocks).
+One step = the selector (sta_build_blocks) plus the block-sparse attention
+(sta_sparse_attn_fwd) on one batch.  --workload picks the other workloads
+(tra_entropy, heta_routed, ab_sampled); a step is then that workload's
+selector plus attention.
 
-  value      effective TFLOP/s on retained blocks (4*d FLOPs per kept query-key
-             pair, true block lengths) per step, inputs resident in HBM
-  e2e        the same metric through the C ABI with host buffers: pinned H2D
-             copies of q, k, v and the D2H copy of o inside the timed region
+Reported (one JSON line on rank 0):
+  value      effective TFLOP/s on retained blocks (4*d FLOPs per kept
+             query-key pair, true block lengths) per step, inputs resident in
+             HBM, summed over ranks
+  e2e        the same metric through the C ABI with pinned host buffers: H2D
+             copies of the step's inputs and the D2H copy of o are inside the
+             timed region
   speedup_vs_dense   dense attention (sta_dense_attn_fwd, same kernel, all
              keys) time / sparse attention time at the same shape
   roofline   the attention kernel against the measured bf16 tensor peak
+  selector   the selector's own time and, where it is bandwidth-bound, its
+             algorithmic bytes against the measured HBM bandwidth
   cpu_baseline  the fp64 oracle on a bounded sample, host cores
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                [--impl reference]
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
 data-path collective); the time is the max over ranks.
 """
@@ -22,7 +31,6 @@ import hashlib
 import json
 import math
 import os
-import subprocess
 import sys
 import threading
 import time
@@ -31,22 +39,28 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "effective TFLOP/s on retained blocks; speedup vs dense at same shape (1×B200)"
-WORKLOAD = "wan_radial"
+DEFAULT_WORKLOAD = "wan_radial"
+WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 * 1024 * 1024
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of attn_fwd.cu, first 16 hex).
-NCU_TRAFFIC = {"source_sha": "61bd247adb317a0a", "bytes_per_launch": 303713280 + 87362304}
+NCU_TRAFFIC = {"source_sha": "61bd247adb317a0a", "workload": "wan_radial",
+               "bytes_per_launch": 303713280 + 87362304}
 
 
-def parse():
+def parse(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--steps", type=int, default=30)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOADS)
     p.add_argument("--no-cpu-baseline", action="store_true")
-    return p.parse_args()
+    p.add_argument("--cpu-budget-s", type=float, default=15.0,
+                   help="seconds of oracle work in the cpu_baseline sample")
+    return p.parse_args(argv)
 
 
 def peaks():
@@ -66,6 +80,9 @@ def source_sha():
 
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML while running."""
+
+    _NAMES = [(0x8, "hw_slowdown"), (0x40, "hw_thermal_slowdown"), (0x20, "sw_thermal_slowdown"),
+              (0x4, "sw_power_cap"), (0x80, "hw_power_brake_slowdown")]
 
     def __init__(self, device_index=0):
         self.samples = []
@@ -93,16 +110,13 @@ class ClockSampler:
         except Exception:
             self._h = None
 
-    _NAMES = [(0x8, "hw_slowdown"), (0x40, "hw_thermal_slowdown"), (0x20, "sw_thermal_slowdown"),
-              (0x4, "sw_power_cap"), (0x80, "hw_power_brake_slowdown")]
-
     def _run(self):
         nv = self._nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
-                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
                 r = fn(self._h)
                 for bit, name in self._NAMES:
                     if r & bit:
@@ -130,100 +144,179 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(s)}
 
 
-def dist_setup(n_gpus):
-    import torch
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+# ------------------------------------------------------------------ ranks
+def rank_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def dist_setup(backend="nccl", timeout_s=120):
+    """One process per GPU; returns (rank, world_size, local_rank)."""
+    rank, ws, local = rank_env()
+    if backend == "nccl":
+        import torch
+        torch.cuda.set_device(local if ws > 1 else 0)
     if ws > 1:
         import datetime
+        import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
+        kw = {}
+        if backend == "nccl":
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
     return rank, ws, local
 
 
 def max_over_ranks(x, ws):
-    import torch
+    """Max of a host float over ranks (NCCL on the device, gloo on the host)."""
     if ws == 1:
-        return x
+        return float(x)
+    import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(ws):
+def sum_over_ranks(x, ws):
+    if ws == 1:
+        return float(x)
     import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(ws, cuda=True):
     if ws > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        import torch
+        torch.cuda.synchronize()
 
 
-def cpu_baseline(w, budget_s=15.0):
-    """Oracle (fp64, numpy) on a bounded sample of the workload: the full radial
-    list build, then attention for query blocks of head 0 until the budget is
-    spent.  Returns the oracle's effective TFLOP/s over the sampled work."""
+# ------------------------------------------------------------ CPU baseline
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return int(max([i.get("num_threads", 1) for i in threadpool_info()] or [1]))
+    except Exception:
+        return 1
+
+
+def cpu_baseline(w, budget_s=15.0, seed=0):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload.
+
+    Per workload: the oracle selector on (a sample of) the rows it needs,
+    then oracle attention for query blocks of head 0 in a seeded order until
+    the budget is spent.  Selector time is charged pro rata to the sampled
+    fraction.  Returns effective TFLOP/s over the sampled retained pairs."""
     import numpy as np
-    from threadpoolctl import threadpool_info
 
-    from oracle import radial
-    from oracle.pipeline import block_sparse_rows
-    from synthetic import make_qkv
+    from oracle import entropy, ibcs_sip, radial, routed
+    from oracle.grid import n_blocks
+    from oracle.pipeline import block_sparse_rows, routed_rows
+    from synthetic import make_difficulty, make_qkv
 
+    N, d, heads = w["N"], w["d"], w["heads"]
+    B, U = w["block_q"], w["kv_unit"]
     q, k, v = make_qkv(dict(w, heads=1))
-    t0 = time.perf_counter()
-    lists = radial.block_lists(w["F"], w["H"], w["W"], w["block_q"], w["radial"])
-    t_sel = time.perf_counter() - t0
-    N, B, d = w["N"], w["block_q"], w["d"]
     qh, kh, vh = (x[0].float().numpy().astype(np.float64) for x in (q, k, v))
-    rng = np.random.default_rng(0)
-    order = rng.permutation(len(lists))
+    rng = np.random.default_rng(seed)
+    nqb = n_blocks(N, B)
+    order = rng.permutation(nqb)
     flops = 0.0
     done = 0
+    t_sel_per_item = 0.0
+    sel = w["selector"]
     t0 = time.perf_counter()
+    if sel == "radial":
+        lists = radial.block_lists(w["F"], w["H"], w["W"], B, w["radial"])
+        t_sel_per_item = (time.perf_counter() - t0) / (nqb * heads)
+        logw = None
+    elif sel == "entropy":
+        e = w["entropy"]
+        lists, _, _, _ = entropy.select(qh, kh, w["F"], w["H"], w["W"], B, e["alpha"], e["beta"],
+                                        e["r_lo"], e["r_hi"], e["tile_h"], e["tile_w"])
+        t_sel_per_item = (time.perf_counter() - t0) / nqb  # one head's selector
+        logw = None
+    elif sel == "routed":
+        c = w["routed"]
+        dif = make_difficulty(w)
+        ids = routed.route(dif, c["dense_frac"])
+        flag = np.zeros(N, bool)
+        flag[ids] = True
+        t_sel_per_item = (time.perf_counter() - t0) / (nqb * heads)
+    elif sel == "ibcs_sip":
+        c = w["ibcs"]
+        kbar, n_j = ibcs_sip.subblock_means(kh, U)
+        t_sel_per_item = (time.perf_counter() - t0) / nqb  # one head's sub-block means
+    budget_end = time.perf_counter() + budget_s
+    t_att = 0.0
     for qb in order:
-        block_sparse_rows(qh, kh, vh, int(qb), lists[qb], B, B)
-        qlen = min(B, N - qb * B)
-        keys = sum(min(B, N - u * B) for u in lists[qb])
-        flops += 4.0 * d * qlen * keys
+        qb = int(qb)
+        ts = time.perf_counter()
+        if sel == "ibcs_sip":
+            lo, hi = qb * B, min(N, qb * B + B)
+            row = ibcs_sip.select_row(qh[lo:hi], kbar, n_j, c["seed"], qb, c["k"], c["iters"],
+                                      c["sample_frac"])
+            block_sparse_rows(qh, kh, vh, qb, row["ids"], B, U, row["logw"])
+            t_att += time.perf_counter() - ts
+            keys = sum(min((u + 1) * U, N) - u * U for u in row["ids"])
+            flops += 4.0 * d * (hi - lo) * keys
+        elif sel == "routed":
+            c = w["routed"]
+            toks = np.arange(qb * B, min(N, qb * B + B))
+            routed_rows(qh, kh, vh, toks, flag, w["F"], w["H"], w["W"], c["win_f"], c["win_h"],
+                        c["win_w"])
+            t_att += time.perf_counter() - ts
+            for t in toks:
+                if flag[t]:
+                    flops += 4.0 * d * N
+                else:
+                    flops += 4.0 * d * len(routed.window_keys(int(t), w["F"], w["H"], w["W"],
+                                                              c["win_f"], c["win_h"],
+                                                              c["win_w"]))
+        else:
+            block_sparse_rows(qh, kh, vh, qb, lists[qb], B, U, logw)
+            t_att += time.perf_counter() - ts
+            qlen = min(B, N - qb * B)
+            keys = sum(min(U, N - u * U) for u in lists[qb])
+            flops += 4.0 * d * qlen * keys
         done += 1
-        if time.perf_counter() - t0 > budget_s:
+        if time.perf_counter() > budget_end:
             break
-    t_att = time.perf_counter() - t0
-    frac = done / (len(lists) * w["heads"])
-    t = t_att + t_sel * frac
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": int(threads),
-            "kind": "oracle",
-            "sample": f"fp64 numpy oracle: full radial list build ({t_sel:.2f} s, charged "
-                      f"pro rata) + attention of {done} of {len(lists) * w['heads']} "
-                      f"(head, query-block) items of head 0, {flops / 1e12:.3f} TFLOP retained",
+    t = t_att + t_sel_per_item * done
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle on {w['name']}: selector charged pro rata "
+                      f"({t_sel_per_item * 1e3:.2f} ms per (head, query-block) item) + "
+                      f"attention of {done} of {nqb * heads} (head, query-block) items of "
+                      f"head 0, {flops / 1e12:.4f} TFLOP retained, {t:.1f} s",
             "host_cpus": os.cpu_count()}
 
 
 def run_reference(args):
-    """The oracle as the reference arm: each step is a bounded sample."""
+    """The oracle as the reference arm: each step is a bounded sample of the
+    workload on the host cores.  Under torchrun rank 0 alone runs it."""
     from synthetic import workload
-    rank = int(os.environ.get("RANK", "0"))
+    rank, ws, _ = rank_env()
     if rank != 0:
         return 0
-    w = workload(WORKLOAD)
+    w = workload(args.workload)
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
-    for _ in range(args.warmup):
-        cpu_baseline(w, budget_s=budget)
-    vals = [cpu_baseline(w, budget_s=budget) for _ in range(args.steps)]
+    for i in range(args.warmup):
+        cpu_baseline(w, budget_s=budget, seed=i)
+    vals = [cpu_baseline(w, budget_s=budget, seed=100 + i) for i in range(args.steps)]
     val = sum(v["value"] for v in vals) / len(vals)
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": {"workload": WORKLOAD, "heads": w["heads"], "F": w["F"], "H": w["H"],
-                       "W": w["W"], "d": w["d"], "block_q": w["block_q"]},
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w),
             "cpu_baseline": dict(vals[-1], value=val),
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -231,33 +324,66 @@ def run_reference(args):
     return 0
 
 
-def main():
-    args = parse()
+def config_of(w):
+    c = {"workload": w["name"], "heads": w["heads"], "F": w["F"], "H": w["H"], "W": w["W"],
+         "N": w["N"], "d": w["d"], "block_q": w["block_q"], "kv_unit": w["kv_unit"],
+         "selector": w["selector"],
+         "l2": f"inputs {3 * w['heads'] * w['N'] * w['d'] * 2 / 1e6:.0f} MB > 126 MB L2; "
+               f"{L2_FLUSH_BYTES >> 20} MB flush write between steps"}
+    return c
+
+
+# ------------------------------------------------------------------- GPU arm
+SELECTOR_LAUNCHES = {"radial": 1, "entropy": 2, "routed": 2, "ibcs_sip": 5}
+
+
+def selector_bytes(w, lists_entries):
+    """Algorithmic bytes of the selector: each input read once plus the list
+    entries written (4 B per id, 4 more per log-weight), and the bound."""
+    h, N, d = w["heads"], w["N"], w["d"]
+    sel = w["selector"]
+    if sel == "entropy":
+        return 2 * h * N * d * 2 + 4 * lists_entries, "hbm"
+    if sel == "ibcs_sip":
+        return 2 * h * N * d * 2 + 8 * lists_entries, "fma (fp32 importance GEMM)"
+    if sel == "routed":
+        return 4 * N + 5 * N + 4 * lists_entries, "latency"
+    return 4 * lists_entries, "launch"
+
+
+def main(argv=None):
+    args = parse(argv)
     if args.impl == "reference":
         return run_reference(args)
     import torch
 
     import sparse_spatiotemporal_attention_video_b200 as sta
     from sparse_spatiotemporal_attention_video_b200 import session
-    from synthetic import make_qkv, workload
+    from synthetic import make_difficulty, make_qkv, workload
 
-    rank, ws, local = dist_setup(args.gpus)
-    w = workload(WORKLOAD)
+    rank, ws, local = dist_setup("nccl")
+    w = workload(args.workload)
     q, k, v = make_qkv(w)
-    prob = session.problem(w)
-    sel = session.selector(w)
-    prm = session.attn_params(w)
+    routed = w["selector"] == "routed"
+    dif = torch.from_numpy(make_difficulty(w)) if routed else None
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    difd = dif.cuda() if routed else None
     od = torch.empty_like(qd)
+    prob = session.problem(w)
+    sel = session.selector(w, difd)
+    prm = session.attn_params(w)
     L = session.Lists(w)
+    sws = session.selector_workspace(w)
+    needs_qk = w["selector"] in ("entropy", "ibcs_sip")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()
-    l2_flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    l2_flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
     def step(qq, kk, vv, oo, ev=None):
         if ev is not None:
             ev[0].record(stream)
-        sta.sta_build_blocks(prob, sel, None, None, L.struct, dev_status=st, stream=stream)
+        sta.sta_build_blocks(prob, sel, qq if needs_qk else None, kk if needs_qk else None,
+                             L.struct, workspace=sws, dev_status=st, stream=stream)
         if ev is not None:
             ev[1].record(stream)
         sta.sta_sparse_attn_fwd(prob, prm, qq, kk, vv, L.struct, oo, dev_status=st,
@@ -270,9 +396,13 @@ def main():
     torch.cuda.synchronize()
     if int(st.item()) != 0:
         raise RuntimeError("device status " + sta.sta_dev_status_string(int(st.item())))
-    pairs = session.retained_pairs(w, L)
+    if routed:
+        pairs = session.retained_pairs_routed(w, L.routed_flag)
+    else:
+        pairs = session.retained_pairs(w, L)
     flops = 4.0 * w["d"] * pairs
     dense_flops = 4.0 * w["d"] * float(w["N"]) ** 2 * w["heads"]
+    entries = int(L.cnt.sum().item())
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier(ws)
@@ -283,16 +413,17 @@ def main():
         torch.cuda.synchronize()
     barrier(ws)
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    sel_ms = [e[0].elapsed_time(e[1]) for e in evs]
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    ms = sum(step_ms) / len(step_ms)
-    ms = max_over_ranks(ms, ws)
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), ws)
+    sel_avg = sum(sel_ms) / len(sel_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
 
     # dense at the same shape (the speedup denominator)
-    for _ in range(3):
+    for _ in range(2):
         sta.sta_dense_attn_fwd(prob, qd, kd, vd, 0.0, od, dev_status=st, stream=stream)
     dense_ms = []
-    for _ in range(max(3, args.steps // 2)):
+    for _ in range(max(3, min(10, args.steps // 3))):
         l2_flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -303,17 +434,17 @@ def main():
     dense_avg = sum(dense_ms) / len(dense_ms)
 
     # end to end through the C ABI with host buffers
-    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    host_in = [x.pin_memory() for x in (q, k, v)] + ([dif.pin_memory()] if routed else [])
+    dev_in = [qd, kd, vd] + ([difd] if routed else [])
     oh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
-    h2d = 3 * qh.numel() * qh.element_size()
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
     d2h = oh.numel() * oh.element_size()
     e2e_ms = []
-    for i in range(args.warmup + max(3, args.steps // 2)):
+    for i in range(args.warmup + max(3, args.steps // 3)):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
+        for hsrc, ddst in zip(host_in, dev_in):
+            ddst.copy_(hsrc, non_blocking=True)
         step(qd, kd, vd, od)
         oh.copy_(od, non_blocking=True)
         b.record(stream)
@@ -326,19 +457,19 @@ def main():
 
     pk, pk_kind = peaks()
     peak = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     achieved = flops / (attn_avg * 1e-3) / 1e12
     traffic = None
-    if NCU_TRAFFIC["source_sha"] and NCU_TRAFFIC["source_sha"] == source_sha():
+    if NCU_TRAFFIC["source_sha"] == source_sha() and NCU_TRAFFIC["workload"] == w["name"]:
         traffic = NCU_TRAFFIC["bytes_per_launch"]
+    sbytes, sbound = selector_bytes(w, entries)
+    sel_gbs = sbytes / (sel_avg * 1e-3) / 1e9
+    total_flops = sum_over_ranks(flops, ws)
     line = {
-        "metric": METRIC, "value": flops * ws / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "metric": METRIC, "value": total_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": WORKLOAD, "heads": w["heads"], "F": w["F"], "H": w["H"],
-                   "W": w["W"], "N": w["N"], "d": w["d"], "block_q": w["block_q"],
-                   "kv_unit": w["kv_unit"], "selector": "radial",
-                   "l2": "inputs 302 MB > 126 MB L2; 256 MB flush write between steps"},
+        "data": "synthetic", "config": config_of(w),
         "retained_pairs": pairs, "retained_fraction": pairs / (w["N"] ** 2 * w["heads"]),
         "attn_ms": attn_avg, "dense_ms": dense_avg,
         "dense_tflops": dense_flops / (dense_avg * 1e-3) / 1e12,
@@ -346,13 +477,16 @@ def main():
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_source": f"{pk_kind} bf16 (burst)"},
-        "e2e": {"value": flops * ws / (e2e_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "selector": {"ms": sel_avg, "bytes": sbytes, "bound": sbound, "achieved_gbs": sel_gbs,
+                     "hbm_peak_gbs": hbm, "frac_of_hbm": sel_gbs / hbm,
+                     "list_entries": entries},
+        "e2e": {"value": total_flops / (e2e_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_avg, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (SELECTOR_LAUNCHES[w["selector"]] + 1) * args.steps,
         "clocks": clk.summary(),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget_s)
     if rank == 0:
         print(json.dumps(line))
     if ws > 1:
