@@ -248,6 +248,13 @@ sta_status sta_sparse_attn_fwd_noalloc(const sta_problem* prob, const sta_attn_p
 const char* sta_status_string(sta_status s);
 const char* sta_dev_status_string(int32_t bits);
 
+/*
+ * Description of the last CUDA error an entry point of this library ran into
+ * on the calling thread (the reason behind a STA_ERR_CUDA return), or "no CUDA
+ * error".  The string is static; the record persists until the next failure.
+ */
+const char* sta_last_cuda_error(void);
+
 /* Library version (major*10000 + minor*100 + patch). */
 int sta_version(void);
 

@@ -86,6 +86,7 @@ SIGNATURES = {
     "sta_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sta_dev_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "sta_version": (ctypes.c_int, []),
+    "sta_last_cuda_error": (ctypes.c_char_p, []),
 }
 
 _lib = None
@@ -113,7 +114,10 @@ class StaError(RuntimeError):
     def __init__(self, code, what):
         self.code = code
         lib = load()
-        super().__init__(f"{what}: {lib.sta_status_string(code).decode()} ({code})")
+        msg = f"{what}: {lib.sta_status_string(code).decode()} ({code})"
+        if code == STA_ERR_CUDA:
+            msg += f": {lib.sta_last_cuda_error().decode()}"
+        super().__init__(msg)
 
 
 def check(code, what):

@@ -13,26 +13,32 @@
 //               128-byte swizzle) into a K ring and a V ring; gathered query
 //               rows (routed items) are copied by the warp and swizzled by
 //               hand.
-//   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM
-//               S buffers (tcgen05.mma, M=128 N=128 K=16 steps, both
-//               operands K-major in shared memory), then O += P V with P
-//               read from TMEM (bf16, aliased onto the S buffer) and V
-//               MN-major in shared memory.  QK of tile t+1 is issued before
-//               PV of tile t, so the tensor core works on the next tile while
-//               the softmax warps handle the current one.
-//   warps 2-9   softmax, two groups of 4 warps: query row r (TMEM lane r)
-//               is shared by one thread of each group, each taking 64 of the
-//               128 logits of a tile: masks partial units / window, adds
-//               log-weights, keeps a running max (exchanged between the two
-//               halves) and a partial sum in registers (max updates that move
-//               by <= 8 in log2 units are deferred, so O in TMEM is rescaled
-//               only on large jumps), writes P as bf16 into TMEM, and finally
-//               normalises its half of O and stores it.  The row sum adds the
-//               bf16-rounded P the tensor core multiplies, not the fp32
-//               values: numerator and denominator then carry the same
-//               weights, so a dominant key's rounding error scales with
-//               (v - O) instead of v (with a deferred maximum its weight is
-//               not exactly 1, and summing fp32 P doubled the output error).
+//   warp 1      MMA issuer (one thread): S = Q K^T of tile t into TMEM S
+//               buffer t%2 (tcgen05.mma, M=128 N=128 K=16 steps, both
+//               operands K-major in shared memory), then O_0 += P[:, 0:64]
+//               V[0:64] and O_1 += P[:, 64:128] V[64:128] with P read from
+//               TMEM (bf16, aliased onto the S buffer) and V MN-major in
+//               shared memory.  QK of tile t+1 is issued before PV of tile t.
+//               TMEM: S_0 | S_1 | O_0 | O_1 (512 columns).
+//   warps 2-9   softmax, two groups of 4 warps.  Group J owns keys
+//               [64J, 64J+64) of every tile and the accumulator O_J: thread r
+//               of the group holds query row r (TMEM lane r), reads its 64
+//               logits, masks partial units / the local window, adds
+//               log-weights, keeps its own running max m_J and sum l_J in
+//               registers (max updates that move by <= 8 in log2 units are
+//               deferred, so O_J is rescaled only on large jumps) and writes
+//               P as bf16 into TMEM.  The two groups never wait on each other
+//               inside an item: each is an independent online softmax over its
+//               half of the keys.  At the end of an item the two (m, l) of a
+//               row are exchanged once through shared memory and each group
+//               writes half of the output columns:
+//                 O = (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)).
+//               The row sum adds the bf16-rounded P the tensor core
+//               multiplies, not the fp32 values: numerator and denominator
+//               then carry the same weights, so a dominant key's rounding
+//               error scales with (v - O) instead of v (with a deferred
+//               maximum its weight is not exactly 1, and summing fp32 P
+//               doubled the output error).
 // Every wait is bounded; a timeout raises STA_DEV_TIMEOUT, sets a CTA-wide
 // abort flag and unwinds without trapping.
 #include <cuda.h>
@@ -79,12 +85,12 @@ struct Layout {
   static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
   // barriers: q_full, q_empty, k_full[KS], k_empty[KS], v_full[VS],
-  // v_empty[VS], s_full[2], p_full[2], o_done[2], mma_done, then the row
-  // exchange barriers of the two softmax groups: xbar[2][4], lbar[4]
-  static constexpr int NBAR = 2 + 2 * KS + 2 * VS + 7 + 12;
+  // v_empty[VS], s_full[2], p_full[2], o_done[2], o_free, mma_done, and the
+  // (m, l) exchange barriers of the two softmax groups: lbar[4]
+  static constexpr int NBAR = 2 + 2 * KS + 2 * VS + 8 + 4;
   static constexpr int OFF_RED = OFF_BAR + NBAR * 8;
-  // red_max[2 parity][2 groups][128 rows], red_l[2 groups][128 rows] (fp32)
-  static constexpr int OFF_MISC = OFF_RED + (2 * 2 * 128 + 2 * 128) * 4;
+  // red_m[2 item parity][2 groups][128 rows], red_l[same] (fp32)
+  static constexpr int OFF_MISC = OFF_RED + 2 * (2 * 2 * 128) * 4;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024
 };
@@ -247,36 +253,93 @@ __device__ __forceinline__ void mask_half(float (&x)[64], const TileInfo<UNIT>& 
 }
 
 struct SoftmaxShared {
-  uint64_t* s_full;
-  uint64_t* p_full;
-  uint64_t* o_done;
-  uint64_t* xbar;   // [2 parity][4 quadrants], 64 arrivals
-  uint64_t* lbar;   // [4 quadrants], 64 arrivals
-  float* red_max;   // [2 parity][2 groups][128 rows]
-  float* red_l;     // [2 groups][128 rows]
+  uint64_t* s_full;  // [2]: S buffer J holds the logits of the current tile of parity J
+  uint64_t* p_full;  // [2]: 256 arrivals, P of the tile in S buffer J is in TMEM
+  uint64_t* o_done;  // [2]: the PV into O_J of the last committed tile has completed
+  uint64_t* o_free;  // 256 arrivals: both O accumulators have been read out
+  uint64_t* lbar;    // [4 quadrants], 64 arrivals: (m, l) exchange of an item
+  float* red_m;      // [2 item parity][2 groups][128 rows]
+  float* red_l;      // [2 item parity][2 groups][128 rows]
   volatile int* abort;
 };
 
 __device__ __forceinline__ float nan_flag() { return __int_as_float(0x7fc00000); }
 
-// Softmax warpgroup WG (4 warps).  Thread (quadrant q, lane l) owns query
-// row r = 32q + l of the tile and, of each 128-key tile, the 64 logits
-// [WG*64, WG*64+64); the partner thread of the other group owns the other
-// half of the same row.  Per tile the two exchange their raw row maxima
-// through shared memory (bounded mbarrier, no bar.sync: a partner that gave
-// up cannot block this one), so both apply the same running maximum; each
-// keeps its own partial row sum, combined in the epilogue.  P (bf16) is
-// written over the group's own logit columns; each group rescales and
-// stores its half of O's columns.
-template <int D, int UNIT, int WG>
+// Exponentials of one 64-column half: p = 2^(x*scale_log2 - m), packed to
+// bf16 pairs; returns the sum of the rounded values.
+__device__ __forceinline__ float exp_pack_half(const float (&x)[64], float scale_log2, float m,
+                                               bool simple, uint32_t (&pk)[32]) {
+  float ls[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) ls[j] = 0.f;
+  if (simple) {
+    // part of the exponentials on the FMA pipe, the rest on MUFU
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+      const float a0 = fmaf(x[c], scale_log2, -m);
+      const float a1 = fmaf(x[c + 1], scale_log2, -m);
+      float p0, p1;
+      if (STA_POLY_EVERY > 0 && ((c >> 1) % (STA_POLY_EVERY > 0 ? STA_POLY_EVERY : 1)) ==
+                                    (STA_POLY_EVERY > 0 ? STA_POLY_EVERY - 1 : 0)) {
+        p0 = exp2_poly(a0);
+        p1 = exp2_poly(a1);
+      } else {
+        p0 = fast_exp2(a0);
+        p1 = fast_exp2(a1);
+      }
+      pk[c >> 1] = pack_bf16x2(p0, p1);
+      ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 64; c += 2) {
+      const float p0 = fast_exp2(fmaf(x[c], scale_log2, -m));
+      const float p1 = fast_exp2(fmaf(x[c + 1], scale_log2, -m));
+      pk[c >> 1] = pack_bf16x2(p0, p1);
+      ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
+    }
+  }
+  return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+}
+
+__device__ __forceinline__ float max64(const float (&x)[64]) {
+  float mv[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) mv[j] = x[j];
+#pragma unroll
+  for (int c = 8; c < 64; ++c) mv[c & 7] = fmaxf(mv[c & 7], x[c]);
+  return fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
+               fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+}
+
+// Loads logit columns [H*64, H*64+64) of S buffer tS for this thread's row.
+template <int H>
+__device__ __forceinline__ void load_half(uint32_t tS, float (&x)[64]) {
+  uint32_t v0[32], v1[32];
+  tmem_ld32(tS + H * 64, v0);
+  tmem_ld32(tS + H * 64 + 32, v1);
+  tmem_wait_ld();
+  tmem_regs_ready(v0);
+  tmem_regs_ready(v1);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    x[i] = __uint_as_float(v0[i]);
+    x[32 + i] = __uint_as_float(v1[i]);
+  }
+}
+
+// Softmax warpgroup J (4 warps): keys [64J, 64J+64) of every tile, query
+// row r = 32*quadrant + lane per thread, accumulator O_J (see the file
+// comment).
+template <int D, int UNIT, int J>
 __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxShared& sh,
                                              uint32_t tmem, int warp, int lane) {
-  constexpr int CB = WG * 64;   // first logit / P column of this group in an S buffer
-  constexpr int OH = D / 2;     // O columns per group
-  constexpr int OB = WG * OH;   // first O column of this group
+  constexpr int OH = D / 2;     // output columns per group
+  constexpr int OB = J * OH;    // first output column of this group
   const int quad = warp & 3;
   const int r = quad * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+  const uint32_t tO = tmem + lane_off + 256 + J * D;
   const float scale_log2 = a.scale_log2;
   const float inv_scale = kLog2e / scale_log2;  // natural-log weight -> raw logit units
   const uint64_t limit = kWaitLimitNs;
@@ -323,6 +386,7 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
     for (int t = 0; t < I.ntiles; ++t) {
       const uint32_t gg = g + t;
       const uint32_t sb = gg & 1;
+      const uint32_t tS = tmem + lane_off + sb * 128;
       // Tile metadata first: its global loads overlap the wait for S.
       TileInfo<kTileK> td;
       TileInfo<UNIT> ti;
@@ -334,53 +398,23 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         load_tile_info<UNIT>(a, I, t, inv_scale, ti);
         simple = ti.full && !ti.bias && !window;
       }
-      const bool okw = mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit);
-      float x[64];
-      float mloc = -INFINITY;
-      if (okw) {
-        tc_fence_after();
-        uint32_t v0[32], v1[32];
-        const uint32_t ts = tmem + lane_off + sb * 128 + CB;
-        tmem_ld32(ts, v0);
-        tmem_ld32(ts + 32, v1);
-        tmem_wait_ld();
-        tmem_regs_ready(v0);
-        tmem_regs_ready(v1);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          x[i] = __uint_as_float(v0[i]);
-          x[32 + i] = __uint_as_float(v1[i]);
-        }
-        if (!simple) {
-          if (dense_like)
-            mask_half<kTileK, WG>(x, td, false, a, 0, 0, 0);
-          else
-            mask_half<UNIT, WG>(x, ti, window, a, fq, hq, wq);
-        }
-        float mv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) mv[j] = x[j];
-#pragma unroll
-        for (int c = 8; c < 64; ++c) mv[c & 7] = fmaxf(mv[c & 7], x[c]);
-        mloc = fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
-                     fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
-      }
-      // exchange the row maximum with the partner thread
-      float* rm = sh.red_max + sb * 256;
-      rm[WG * 128 + r] = okw ? mloc : nan_flag();
-      mbar_arrive(sh.xbar + sb * 4 + quad);
-      const bool okx = mbar_wait(sh.xbar + sb * 4 + quad, (gg >> 1) & 1, abort, limit);
-      const float mo = rm[(1 - WG) * 128 + r];
-      if (!okw || !okx || mo != mo) {
+      if (!mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit)) {
         ok = false;
         break;
       }
-      const float m_tile = fmaxf(mloc, mo) * scale_log2;  // -inf if all masked
+      tc_fence_after();
+      float x[64];
+      load_half<J>(tS, x);
+      if (!simple) {
+        if (dense_like) mask_half<kTileK, J>(x, td, false, a, 0, 0, 0);
+        else mask_half<UNIT, J>(x, ti, window, a, fq, hq, wq);
+      }
+      const float m_tile = max64(x) * scale_log2;  // -inf if all masked
       const float m_new = fmaxf(m_run, m_tile);
       const bool need = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
       if (__any_sync(0xffffffffu, need)) {
-        // O rows of this warp hold tiles < t; the last of them must be
-        // accumulated before it is rescaled.
+        // O_J holds tiles < t of this item; the last of them (tile gg - 1)
+        // must be accumulated before O_J is rescaled.
         const uint32_t gp = gg - 1;
         if (!mbar_wait(sh.o_done + (gp & 1), (gp >> 1) & 1, abort, limit)) {
           ok = false;
@@ -389,15 +423,14 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         tc_fence_after();
         const float f = need ? fast_exp2(m_run - m_new) : 1.f;
 #pragma unroll
-        for (int ch = 0; ch < OH / 32; ++ch) {
+        for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t v[32];
-          const uint32_t to = tmem + lane_off + 256 + OB + ch * 32;
-          tmem_ld32(to, v);
+          tmem_ld32(tO + ch * 32, v);
           tmem_wait_ld();
           tmem_regs_ready(v);
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-          tmem_st32(to, v);
+          tmem_st32(tO + ch * 32, v);
         }
         tmem_wait_st();
         if (need) {
@@ -407,93 +440,81 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       }
       if (m_run == -INFINITY) m_run = m_new;
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float ls[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) ls[j] = 0.f;
+      // P of this group's 64 keys, packed over the first 32 of its (already
+      // read) logit columns
       uint32_t pk[32];
-      if (simple) {
-        // part of the exponentials on the FMA pipe, the rest on MUFU
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float a0 = fmaf(x[c], scale_log2, -m_use);
-          const float a1 = fmaf(x[c + 1], scale_log2, -m_use);
-          float p0, p1;
-          if (STA_POLY_EVERY > 0 && ((c >> 1) % (STA_POLY_EVERY > 0 ? STA_POLY_EVERY : 1)) ==
-                                        (STA_POLY_EVERY > 0 ? STA_POLY_EVERY - 1 : 0)) {
-            p0 = exp2_poly(a0);
-            p1 = exp2_poly(a1);
-          } else {
-            p0 = fast_exp2(a0);
-            p1 = fast_exp2(a1);
-          }
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-          ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = fast_exp2(fmaf(x[c], scale_log2, -m_use));
-          const float p1 = fast_exp2(fmaf(x[c + 1], scale_log2, -m_use));
-          pk[c >> 1] = pack_bf16x2(p0, p1);
-          ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
-        }
-      }
-      l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      tmem_st32(tmem + lane_off + sb * 128 + CB, pk);
+      l_run += exp_pack_half(x, scale_log2, m_use, simple, pk);
+      tmem_st32(tS + J * 64, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(sh.p_full + sb);
     }
     if (!ok) break;
     // ------------------------------------------------------------ epilogue
-    const uint32_t gl = g + I.ntiles - 1;
-    const bool okw = mbar_wait(sh.o_done + (gl & 1), (gl >> 1) & 1, abort, limit);
-    g += I.ntiles;
-    sh.red_l[WG * 128 + r] = okw ? l_run : nan_flag();
+    const uint32_t gl = g + I.ntiles - 1;  // last tile of the item
+    // (m, l) slots alternate with the item parity: the partner may still be
+    // reading the previous item's slot when this group gets here.
+    const int slot = (nitem & 1) * 256;
+    sh.red_m[slot + J * 128 + r] = m_run;
+    sh.red_l[slot + J * 128 + r] = l_run;
     mbar_arrive(sh.lbar + quad);
-    const bool okx = mbar_wait(sh.lbar + quad, nitem & 1, abort, limit);
+    bool okw = mbar_wait(sh.lbar + quad, nitem & 1, abort, limit);
+    const float mo = sh.red_m[slot + (1 - J) * 128 + r];
+    const float lo = sh.red_l[slot + (1 - J) * 128 + r];
+    // the commit after the item's last PV covers every earlier MMA
+    if (okw) okw = mbar_wait(sh.o_done + (gl & 1), (gl >> 1) & 1, abort, limit);
+    g += I.ntiles;
     ++nitem;
-    const float lo = sh.red_l[(1 - WG) * 128 + r];
-    if (!okw || !okx || lo != lo) {
+    if (!okw) {
       ok = false;
       break;
     }
     tc_fence_after();
-    const float l_tot = l_run + lo;
+    const float m0 = J == 0 ? m_run : mo, m1 = J == 0 ? mo : m_run;
+    const float l0 = J == 0 ? l_run : lo, l1 = J == 0 ? lo : l_run;
+    const float m = fmaxf(m0, m1);
+    const float f0 = (m0 != -INFINITY) ? fast_exp2(m0 - m) : 0.f;
+    const float f1 = (m1 != -INFINITY) ? fast_exp2(m1 - m) : 0.f;
+    const float l_tot = l0 * f0 + l1 * f1;
     const bool empty = !(l_tot > 0.f);
     const float inv_l = empty ? 0.f : 1.f / l_tot;
-    if (WG == 0 && active && empty) raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
+    const float c0 = f0 * inv_l, c1 = f1 * inv_l;
+    if (J == 0 && active && empty) raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
 #pragma unroll
     for (int ch = 0; ch < OH / 32; ++ch) {
+      const uint32_t col = tmem + lane_off + 256 + OB + ch * 32;
+      float o[32];
       uint32_t v[32];
-      tmem_ld32(tmem + lane_off + 256 + OB + ch * 32, v);
+      tmem_ld32(col, v);
       tmem_wait_ld();
       tmem_regs_ready(v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = __uint_as_float(v[i]) * c0;
+      tmem_ld32(col + D, v);
+      tmem_wait_ld();
+      tmem_regs_ready(v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = fmaf(__uint_as_float(v[i]), c1, o[i]);
       if (active) {
-        const size_t col = orow * D + OB + ch * 32;
+        const size_t gcol = orow * D + OB + ch * 32;
         if (a.out_f32) {
-          float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.o) + col);
+          float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.o) + gcol);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            op[i] = make_float4(
-                __uint_as_float(v[4 * i]) * inv_l, __uint_as_float(v[4 * i + 1]) * inv_l,
-                __uint_as_float(v[4 * i + 2]) * inv_l, __uint_as_float(v[4 * i + 3]) * inv_l);
+            op[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         } else {
-          uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + col);
+          uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + gcol);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            op[i] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * i]) * inv_l,
-                                           __uint_as_float(v[8 * i + 1]) * inv_l),
-                               pack_bf16x2(__uint_as_float(v[8 * i + 2]) * inv_l,
-                                           __uint_as_float(v[8 * i + 3]) * inv_l),
-                               pack_bf16x2(__uint_as_float(v[8 * i + 4]) * inv_l,
-                                           __uint_as_float(v[8 * i + 5]) * inv_l),
-                               pack_bf16x2(__uint_as_float(v[8 * i + 6]) * inv_l,
-                                           __uint_as_float(v[8 * i + 7]) * inv_l));
+            op[i] = make_uint4(pack_bf16x2(o[8 * i], o[8 * i + 1]),
+                               pack_bf16x2(o[8 * i + 2], o[8 * i + 3]),
+                               pack_bf16x2(o[8 * i + 4], o[8 * i + 5]),
+                               pack_bf16x2(o[8 * i + 6], o[8 * i + 7]));
         }
       }
     }
     tc_fence_before();
+    mbar_arrive(sh.o_free);
   }
   if (!ok) fail(abort, a.dev_status);
 }
@@ -523,11 +544,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = v_empty + VS;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
-  uint64_t* mma_done = o_done + 2;
-  uint64_t* xbar = mma_done + 1;  // [2][4]
-  uint64_t* lbar = xbar + 8;      // [4]
-  float* red_max = reinterpret_cast<float*>(smem + L::OFF_RED);
-  float* red_l = red_max + 2 * 2 * 128;
+  uint64_t* o_free = o_done + 2;
+  uint64_t* mma_done = o_free + 1;
+  uint64_t* lbar = mma_done + 1;  // [4]
+  float* red_m = reinterpret_cast<float*>(smem + L::OFF_RED);
+  float* red_l = red_m + 2 * 2 * 128;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -547,11 +568,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 256);
+      mbar_init(p_full + i, 256);  // both softmax groups write P of every tile
       mbar_init(o_done + i, 1);
     }
+    mbar_init(o_free, 256);
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(xbar + i, 64);
     for (int i = 0; i < 4; ++i) mbar_init(lbar + i, 64);
     *abort = 0;
     fence_barrier_init();
@@ -674,28 +695,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t tS0 = tmem, tS1 = tmem + 128, tO = tmem + 256;
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       uint32_t kt = 0, vt = 0, qn = 0, g = 0;
       bool ok = true;
-      auto issue_pv = [&](uint32_t gg, bool first) -> bool {
+      // first: the next PV starts the accumulators O_0 / O_1 of this item;
+      // wait_free: O_0/O_1 still hold the previous item until both softmax
+      // groups have read them out (o_free).
+      bool first = true;
+      bool wait_free = false;
+      auto issue_pv = [&](uint32_t gg) -> bool {
         const uint32_t sb = gg & 1;
         if (!mbar_wait(p_full + sb, (gg >> 1) & 1, abort, limit)) return false;
+        if (wait_free) {
+          if (!mbar_wait(o_free, (qn - 1) & 1, abort, limit)) return false;
+          wait_free = false;
+        }
         tc_fence_after();
         const int st = vt % VS;
         if (!mbar_wait(v_full + st, (vt / VS) & 1, abort, limit)) return false;
         tc_fence_after();
-        const uint32_t tS = sb ? tS1 : tS0;
+        const uint32_t tS = tmem + sb * 128;
         const uint32_t vbase = aV + st * L::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
           const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024);
-          // P of keys 0..63 sits in columns 0..31 of the S buffer, keys
-          // 64..127 in columns 64..95 (each softmax group writes over its
-          // own logits)
+          // keys 0..63 (softmax group 0): P in columns 0..31, into O_0;
+          // keys 64..127 (group 1): P in columns 64..95, into O_1
           const uint32_t pa = tS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
-          mma_bf16_ts(tO, pa, bdesc, IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          const uint32_t tO = tmem + 256 + (kk < 4 ? 0 : D);
+          mma_bf16_ts(tO, pa, bdesc, IDESC_PV, (first && (kk & 3) == 0) ? 0u : 1u);
         }
+        first = false;
         mma_commit(v_empty + st);
         ++vt;
         mma_commit(o_done + sb);
@@ -710,6 +740,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
+        first = true;
+        wait_free = qn > 0;
         for (int t = 0; t < I.ntiles; ++t) {
           const int st = kt % KS;
           if (!mbar_wait(k_full + st, (kt / KS) & 1, abort, limit)) {
@@ -718,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sb = (g + t) & 1;
-          const uint32_t tS = sb ? tS1 : tS0;
+          const uint32_t tS = tmem + sb * 128;
           const uint32_t kbase = aK + st * L::TILE_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -731,13 +763,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++kt;
           mma_commit(s_full + sb);
           if (t == I.ntiles - 1) mma_commit(q_empty);
-          if (t > 0 && !issue_pv(g + t - 1, t == 1)) {
+          if (t > 0 && !issue_pv(g + t - 1)) {
             ok = false;
             break;
           }
         }
         if (!ok) break;
-        if (!issue_pv(g + I.ntiles - 1, I.ntiles == 1)) {
+        if (!issue_pv(g + I.ntiles - 1)) {
           ok = false;
           break;
         }
@@ -752,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------- softmax
-    SoftmaxShared sh{s_full, p_full, o_done, xbar, lbar, red_max, red_l, abort};
+    SoftmaxShared sh{s_full, p_full, o_done, o_free, lbar, red_m, red_l, abort};
     if (warp < 6)
       softmax_role<D, UNIT, 0>(a, sh, tmem, warp, lane);
     else

@@ -6,7 +6,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/sta.h"
+#include "sta.h"
 
 namespace sta {
 

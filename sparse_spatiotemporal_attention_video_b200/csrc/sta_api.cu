@@ -16,6 +16,15 @@ namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
 
+// Last CUDA error a call of this thread ran into (sta_last_cuda_error).
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+bool failed(cudaError_t e) {
+  if (e == cudaSuccess) return false;
+  g_last_cuda_error = e;
+  return true;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -94,9 +103,9 @@ sta_status stage_inputs(const sta_problem* p, const void* q, const void* k, cons
   __nv_bfloat16* dq = base;
   __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(ws) + one);
   __nv_bfloat16* dv = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(ws) + 2 * one);
-  if (launch_f32_to_bf16(static_cast<const float*>(q), dq, n, stream) != cudaSuccess ||
-      launch_f32_to_bf16(static_cast<const float*>(k), dk, n, stream) != cudaSuccess ||
-      launch_f32_to_bf16(static_cast<const float*>(v), dv, n, stream) != cudaSuccess)
+  if (failed(launch_f32_to_bf16(static_cast<const float*>(q), dq, n, stream)) ||
+      failed(launch_f32_to_bf16(static_cast<const float*>(k), dk, n, stream)) ||
+      failed(launch_f32_to_bf16(static_cast<const float*>(v), dv, n, stream)))
     return STA_ERR_CUDA;
   *qb = dq;
   *kb = dk;
@@ -113,13 +122,15 @@ sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16*
       !make_map(&tku, kb, p->d, N, p->heads, unit) ||
       !make_map(&tvu, vb, p->d, N, p->heads, unit) ||
       !make_map(&tkf, kb, p->d, N, p->heads, kTileK) ||
-      !make_map(&tvf, vb, p->d, N, p->heads, kTileK))
+      !make_map(&tvf, vb, p->d, N, p->heads, kTileK)) {
+    g_last_cuda_error = cudaErrorInvalidValue;
     return STA_ERR_CUDA;
+  }
   const int sms = num_sms_current();
   if (sms <= 0) return STA_ERR_CUDA;
   a.unit = unit;
   a.q = qb;
-  if (launch_attention(p->d, a, tq, tku, tvu, tkf, tvf, sms, stream) != cudaSuccess)
+  if (failed(launch_attention(p->d, a, tq, tku, tvu, tkf, tvf, sms, stream)))
     return STA_ERR_CUDA;
   return STA_OK;
 }
@@ -171,6 +182,10 @@ int fraction_count(double frac, long long n, int lo) {
 extern "C" {
 
 int sta_version(void) { return kVersion; }
+
+const char* sta_last_cuda_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 const char* sta_status_string(sta_status s) {
   switch (s) {
@@ -228,9 +243,9 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       const int S = prob->H * prob->W;
       if ((sel->block_q + S - 1) / S + 1 > 8) return STA_ERR_UNSUPPORTED;
       out->head_shared = 1;
-      if (launch_radial_lists(prob->F, prob->H, prob->W, sel->block_q, sel->radial_w0,
+      if (failed(launch_radial_lists(prob->F, prob->H, prob->W, sel->block_q, sel->radial_w0,
                               sel->radial_w_off, sel->radial_full_df, out->idx, out->cnt, out->cap,
-                              out->required_cap, dev_status, s) != cudaSuccess)
+                              out->required_cap, dev_status, s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }
@@ -249,15 +264,15 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       float* kbar = reinterpret_cast<float*>(ws + w.kbar);
       out->head_shared = 0;
       const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
-      if (launch_block_means(static_cast<const __nv_bfloat16*>(q),
+      if (failed(launch_block_means(static_cast<const __nv_bfloat16*>(q),
                              static_cast<const __nv_bfloat16*>(k), qbar, kbar, prob->heads, N,
-                             prob->d, sel->block_q, s) != cudaSuccess)
+                             prob->d, sel->block_q, s)))
         return STA_ERR_CUDA;
-      if (launch_entropy_lists(qbar, kbar, prob->heads, prob->F, prob->H, prob->W, prob->d,
+      if (failed(launch_entropy_lists(qbar, kbar, prob->heads, prob->F, prob->H, prob->W, prob->d,
                                sel->block_q, scale, sel->ent_alpha, sel->ent_beta, sel->ent_r_lo,
                                sel->ent_r_hi, sel->ent_tile_h, sel->ent_tile_w, out->idx,
                                out->cnt, out->cap, out->required_cap, out->entropy, out->radius,
-                               dev_status, s) != cudaSuccess)
+                               dev_status, s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }
@@ -269,12 +284,12 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       const int n_routed = fraction_count(sel->dense_frac, N, 0);
       out->head_shared = 1;
       out->n_routed = n_routed;
-      if (launch_routed_select(sel->difficulty, N, n_routed, out->routed_ids, out->routed_flag,
-                               s) != cudaSuccess)
+      if (failed(launch_routed_select(sel->difficulty, N, n_routed, out->routed_ids, out->routed_flag,
+                               s)))
         return STA_ERR_CUDA;
-      if (launch_routed_local_lists(prob->F, prob->H, prob->W, sel->block_q, sel->kv_unit,
+      if (failed(launch_routed_local_lists(prob->F, prob->H, prob->W, sel->block_q, sel->kv_unit,
                                     sel->win_f, sel->win_h, sel->win_w, out->idx, out->cnt,
-                                    out->cap, out->required_cap, dev_status, s) != cudaSuccess)
+                                    out->cap, out->required_cap, dev_status, s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }
@@ -297,13 +312,13 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       out->head_shared = 0;
       const int m = fraction_count(sel->sample_frac, n_sub, 1);
       const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
-      if (launch_block_means(static_cast<const __nv_bfloat16*>(k), nullptr, kbar, nullptr,
-                             prob->heads, N, prob->d, sel->kv_unit, s) != cudaSuccess)
+      if (failed(launch_block_means(static_cast<const __nv_bfloat16*>(k), nullptr, kbar, nullptr,
+                             prob->heads, N, prob->d, sel->kv_unit, s)))
         return STA_ERR_CUDA;
-      if (launch_ibcs_sip(static_cast<const __nv_bfloat16*>(q), kbar, cent, wts, pbuf,
+      if (failed(launch_ibcs_sip(static_cast<const __nv_bfloat16*>(q), kbar, cent, wts, pbuf,
                           prob->heads, N, prob->d, sel->block_q, sel->kv_unit, sel->km_k,
                           sel->km_iters, m, sel->seed, scale, out->idx, out->logw, out->cnt,
-                          out->cap, out->required_cap, dev_status, s) != cudaSuccess)
+                          out->cap, out->required_cap, dev_status, s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }
@@ -433,12 +448,12 @@ void* g_static_stage_ptr[kMaxStaticDevices] = {};
 // first call per device).
 sta_status static_stage_address(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return STA_ERR_CUDA;
+  if (failed(cudaGetDevice(&dev))) return STA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxStaticDevices) return STA_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_static_stage_mu);
   if (!g_static_stage_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_stage) != cudaSuccess || !p) return STA_ERR_CUDA;
+    if (failed(cudaGetSymbolAddress(&p, g_static_stage)) || !p) return STA_ERR_CUDA;
     g_static_stage_ptr[dev] = p;
   }
   *out = g_static_stage_ptr[dev];
