@@ -177,61 +177,66 @@ __device__ __forceinline__ void fail(volatile int* abort, int32_t* st) {
   raise_status(st, STA_DEV_TIMEOUT);
 }
 
-// Per-slot information of one tile for the softmax threads.
+// One softmax group's 64 logit columns of a tile, as SLOTS runs of
+// W = min(UNIT, 64) columns; a 128-key unit contributes the half the group
+// owns.  All per-column indices below are compile-time.
 template <int UNIT>
-struct TileInfo {
-  static constexpr int UPT = kTileK / UNIT;
-  int nv[UPT];
-  float braw[UPT];   // log-weight / scale: added to raw logits
-  int base[UPT];     // first token of the unit
+struct HalfInfo {
+  static constexpr int W = UNIT < 64 ? UNIT : 64;
+  static constexpr int SLOTS = 64 / W;
+  int lim[SLOTS];     // valid columns of the slot (keys past N / empty slots masked)
+  float braw[SLOTS];  // log-weight / scale: added to raw logits
+  int tok0[SLOTS];    // key token of the slot's first column
   bool full, bias;
 };
 
 template <int UNIT>
-__device__ __forceinline__ void load_tile_info(const AttnArgs& a, const Item& I, int t,
-                                               float inv_scale, TileInfo<UNIT>& ti) {
-  ti.full = true;
-  ti.bias = (a.logw != nullptr) && (I.kind == kItemList || I.kind == kItemLocal);
+__device__ __forceinline__ void load_half_info(const AttnArgs& a, const Item& I, int t, int J,
+                                               float inv_scale, HalfInfo<UNIT>& hi) {
+  constexpr int W = HalfInfo<UNIT>::W;
+  hi.full = true;
+  hi.bias = (a.logw != nullptr) && (I.kind == kItemList || I.kind == kItemLocal);
 #pragma unroll
-  for (int s = 0; s < TileInfo<UNIT>::UPT; ++s) {
+  for (int s = 0; s < HalfInfo<UNIT>::SLOTS; ++s) {
+    const int col = J * 64 + s * W;  // first tile column of the slot
+    const int gs = col / UNIT;       // the tile's slot (list position)
+    const int off = col - gs * UNIT;  // column offset inside that unit
     int nv;
     float lw;
     bool bad;
-    const int u = slot_unit(a, I, t, s, nv, lw, bad);
-    ti.nv[s] = nv;
-    ti.braw[s] = lw * inv_scale;
-    ti.base[s] = u * UNIT;
-    if (nv < UNIT) ti.full = false;
+    const int u = slot_unit(a, I, t, gs, nv, lw, bad);
+    const int lim = min(max(nv - off, 0), W);
+    hi.lim[s] = lim;
+    hi.braw[s] = lw * inv_scale;
+    hi.tok0[s] = u * UNIT + off;
+    if (lim < W) hi.full = false;
   }
 }
 
-// Masks (partial units, key tokens past N), log-weights and the local
-// window for the 64 logit columns [WG*64, WG*64+64) one softmax group owns.
-template <int UNIT, int WG>
-__device__ __forceinline__ void mask_half(float (&x)[64], const TileInfo<UNIT>& ti, bool window,
+// Masks (partial units, key tokens past N), log-weights and the local window
+// on one group's 64 logit columns.
+template <int UNIT>
+__device__ __forceinline__ void mask_half(float (&x)[64], const HalfInfo<UNIT>& hi, bool window,
                                           const AttnArgs& a, int fq, int hq, int wq) {
-  constexpr int CB = WG * 64;
-  if (!ti.full) {
+  constexpr int W = HalfInfo<UNIT>::W;
+  if (!hi.full) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      const int cc = CB + c;
-      if ((cc % UNIT) >= ti.nv[cc / UNIT]) x[c] = -INFINITY;
-    }
+    for (int c = 0; c < 64; ++c)
+      if ((c % W) >= hi.lim[c / W]) x[c] = -INFINITY;
   }
-  if (ti.bias) {
+  if (hi.bias) {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) x[c] += ti.braw[(CB + c) / UNIT];
+    for (int c = 0; c < 64; ++c) x[c] += hi.braw[c / W];
   }
   if (window) {
     // key coordinates advance column by column; they are recomputed from the
-    // unit's first token at every unit boundary (all indices compile-time)
+    // slot's first token at every slot boundary
     const int S = a.H * a.W;
     int f = 0, h = 0, w = 0;
 #pragma unroll
     for (int c = 0; c < 64; ++c) {
-      const int cc = CB + c;
-      if (c == 0 || (cc % UNIT) == 0) {
-        const int t0 = ti.base[cc / UNIT] + (cc % UNIT);
+      if ((c % W) == 0) {
+        const int t0 = hi.tok0[c / W];
         f = t0 / S;
         const int rem = t0 - f * S;
         h = rem / a.W;
@@ -266,40 +271,41 @@ struct SoftmaxShared {
 __device__ __forceinline__ float nan_flag() { return __int_as_float(0x7fc00000); }
 
 // Exponentials of one 64-column half: p = 2^(x*scale_log2 - m), packed to
-// bf16 pairs; returns the sum of the rounded values.
+// bf16 pairs; returns the sum of the rounded values.  The scale-and-shift and
+// the running sums use the paired fp32 instructions (two lanes of work per
+// instruction).
 __device__ __forceinline__ float exp_pack_half(const float (&x)[64], float scale_log2, float m,
                                                bool simple, uint32_t (&pk)[32]) {
-  float ls[8];
+  const float2 sl = make_float2(scale_log2, scale_log2);
+  const float2 nm = make_float2(-m, -m);
+  float2 acc[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) ls[j] = 0.f;
-  if (simple) {
-    // part of the exponentials on the FMA pipe, the rest on MUFU
+  for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-      const float a0 = fmaf(x[c], scale_log2, -m);
-      const float a1 = fmaf(x[c + 1], scale_log2, -m);
-      float p0, p1;
-      if (STA_POLY_EVERY > 0 && ((c >> 1) % (STA_POLY_EVERY > 0 ? STA_POLY_EVERY : 1)) ==
-                                    (STA_POLY_EVERY > 0 ? STA_POLY_EVERY - 1 : 0)) {
-        p0 = exp2_poly(a0);
-        p1 = exp2_poly(a1);
-      } else {
-        p0 = fast_exp2(a0);
-        p1 = fast_exp2(a1);
-      }
-      pk[c >> 1] = pack_bf16x2(p0, p1);
-      ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
+  for (int c = 0; c < 64; c += 2) {
+    const float2 arg = __ffma2_rn(make_float2(x[c], x[c + 1]), sl, nm);
+    float p0, p1;
+#if STA_POLY_EVERY > 0
+    // one pair in every STA_POLY_EVERY on the FMA pipe (finite arguments only)
+    if (simple && ((c >> 1) % STA_POLY_EVERY) == STA_POLY_EVERY - 1) {
+      p0 = exp2_poly(arg.x);
+      p1 = exp2_poly(arg.y);
+    } else {
+      p0 = fast_exp2(arg.x);
+      p1 = fast_exp2(arg.y);
     }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 64; c += 2) {
-      const float p0 = fast_exp2(fmaf(x[c], scale_log2, -m));
-      const float p1 = fast_exp2(fmaf(x[c + 1], scale_log2, -m));
-      pk[c >> 1] = pack_bf16x2(p0, p1);
-      ls[(c >> 1) & 7] += bf16_lo(pk[c >> 1]) + bf16_hi(pk[c >> 1]);
-    }
+#else
+    (void)simple;
+    p0 = fast_exp2(arg.x);
+    p1 = fast_exp2(arg.y);
+#endif
+    pk[c >> 1] = pack_bf16x2(p0, p1);
+    acc[(c >> 1) & 3] =
+        __fadd2_rn(acc[(c >> 1) & 3], make_float2(bf16_lo(pk[c >> 1]), bf16_hi(pk[c >> 1])));
   }
-  return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+  const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 t = __fadd2_rn(s01, s23);
+  return t.x + t.y;
 }
 
 __device__ __forceinline__ float max64(const float (&x)[64]) {
@@ -312,12 +318,11 @@ __device__ __forceinline__ float max64(const float (&x)[64]) {
                fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
 }
 
-// Loads logit columns [H*64, H*64+64) of S buffer tS for this thread's row.
-template <int H>
-__device__ __forceinline__ void load_half(uint32_t tS, float (&x)[64]) {
+// Loads 64 consecutive TMEM columns starting at taddr (this thread's lane).
+__device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
   uint32_t v0[32], v1[32];
-  tmem_ld32(tS + H * 64, v0);
-  tmem_ld32(tS + H * 64 + 32, v1);
+  tmem_ld32(taddr, v0);
+  tmem_ld32(taddr + 32, v1);
   tmem_wait_ld();
   tmem_regs_ready(v0);
   tmem_regs_ready(v1);
@@ -331,11 +336,11 @@ __device__ __forceinline__ void load_half(uint32_t tS, float (&x)[64]) {
 // Softmax warpgroup J (4 warps): keys [64J, 64J+64) of every tile, query
 // row r = 32*quadrant + lane per thread, accumulator O_J (see the file
 // comment).
-template <int D, int UNIT, int J>
+template <int D, int UNIT>
 __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxShared& sh,
-                                             uint32_t tmem, int warp, int lane) {
+                                             uint32_t tmem, int warp, int lane, int J) {
   constexpr int OH = D / 2;     // output columns per group
-  constexpr int OB = J * OH;    // first output column of this group
+  const int OB = J * OH;        // first output column of this group
   const int quad = warp & 3;
   const int r = quad * 32 + lane;
   const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -388,14 +393,14 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       const uint32_t sb = gg & 1;
       const uint32_t tS = tmem + lane_off + sb * 128;
       // Tile metadata first: its global loads overlap the wait for S.
-      TileInfo<kTileK> td;
-      TileInfo<UNIT> ti;
+      HalfInfo<kTileK> td;
+      HalfInfo<UNIT> ti;
       bool simple;  // no masked column, no weight, no window
       if (dense_like) {
-        load_tile_info<kTileK>(a, I, t, inv_scale, td);
+        load_half_info<kTileK>(a, I, t, J, inv_scale, td);
         simple = td.full;
       } else {
-        load_tile_info<UNIT>(a, I, t, inv_scale, ti);
+        load_half_info<UNIT>(a, I, t, J, inv_scale, ti);
         simple = ti.full && !ti.bias && !window;
       }
       if (!mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit)) {
@@ -404,10 +409,10 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       }
       tc_fence_after();
       float x[64];
-      load_half<J>(tS, x);
+      load_cols64(tS + J * 64, x);
       if (!simple) {
-        if (dense_like) mask_half<kTileK, J>(x, td, false, a, 0, 0, 0);
-        else mask_half<UNIT, J>(x, ti, window, a, fq, hq, wq);
+        if (dense_like) mask_half<kTileK>(x, td, false, a, 0, 0, 0);
+        else mask_half<UNIT>(x, ti, window, a, fq, hq, wq);
       }
       const float m_tile = max64(x) * scale_log2;  // -inf if all masked
       const float m_new = fmaxf(m_run, m_tile);
@@ -785,10 +790,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------- softmax
     SoftmaxShared sh{s_full, p_full, o_done, o_free, lbar, red_m, red_l, abort};
-    if (warp < 6)
-      softmax_role<D, UNIT, 0>(a, sh, tmem, warp, lane);
-    else
-      softmax_role<D, UNIT, 1>(a, sh, tmem, warp, lane);
+    // one copy of the softmax code serves both groups (J is a runtime value)
+    softmax_role<D, UNIT>(a, sh, tmem, warp, lane, warp < 6 ? 0 : 1);
   }
 
   tc_fence_before();
