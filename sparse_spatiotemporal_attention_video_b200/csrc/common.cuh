@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "sta.h"
 
 namespace sta {
@@ -69,6 +71,26 @@ cudaError_t launch_radial_lists(int F, int H, int W, int B, int w0, int w_off, i
                                 int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
                                 int32_t* dev_status, cudaStream_t stream);
 
+// Raises kernel Fn's dynamic shared memory limit to at least `bytes` on the
+// current device, calling cudaFuncSetAttribute only when the limit grows (the
+// attribute is per device, and the call costs host time on every launch).
+template <auto Fn>
+cudaError_t set_dyn_smem(int bytes) {
+  static std::atomic<int> done[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < 64;
+  if (cached && done[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(Fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) {
+    int prev = done[dev].load(std::memory_order_relaxed);
+    while (prev < bytes && !done[dev].compare_exchange_weak(prev, bytes)) {
+    }
+  }
+  return e;
+}
+
 // Block means (sel_pool.cu): out_i[h][b][d] = mean of the rows of block b of
 // x_i (fp32); x1/out1 may be null.
 cudaError_t launch_block_means(const __nv_bfloat16* x0, const __nv_bfloat16* x1, float* out0,
@@ -76,11 +98,12 @@ cudaError_t launch_block_means(const __nv_bfloat16* x0, const __nv_bfloat16* x1,
 
 // Entropy-radius selector (sel_entropy.cu).
 int entropy_max_blocks(int d);
-cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, int heads, int F, int H,
-                                 int W, int d, int B, float scale, float alpha, float beta,
-                                 int r_lo, int r_hi, int tile_h, int tile_w, int32_t* idx,
-                                 int32_t* cnt, int cap, int32_t* required_cap, float* entropy,
-                                 int32_t* radius, int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, float* scores, int heads,
+                                 int F, int H, int W, int d, int B, float scale, float alpha,
+                                 float beta, int r_lo, int r_hi, int tile_h, int tile_w,
+                                 int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
+                                 float* entropy, int32_t* radius, int32_t* dev_status,
+                                 cudaStream_t s);
 
 // Difficulty routing (sel_routed.cu).
 cudaError_t launch_routed_select(const float* difficulty, int N, int n_routed,
@@ -93,7 +116,7 @@ cudaError_t launch_routed_local_lists(int F, int H, int W, int B, int U, int win
 // Clustering importance + inclusion-probability sampling (sel_ibcs.cu).
 int ibcs_max_subblocks();
 cudaError_t launch_ibcs_sip(const __nv_bfloat16* q, const float* kbar, float* cent, float* wts,
-                            float* p, int heads, int N, int d, int B, int U, int km_k, int iters,
+                            float* z, float* stats, int heads, int N, int d, int B, int U, int km_k, int iters,
                             int m, uint64_t seed, float scale, int32_t* idx, float* logw,
                             int32_t* cnt, int cap, int32_t* required_cap, int32_t* dev_status,
                             cudaStream_t s);

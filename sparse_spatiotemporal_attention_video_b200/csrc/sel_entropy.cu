@@ -22,11 +22,15 @@
 // the radius map use explicit round-to-nearest operations (no FMA
 // contraction), as the decision is defined on them.
 //
-// One CTA of 8 warps handles 8 query blocks of one head: pooled key blocks
-// are staged in shared memory in chunks of 64 (rows padded to D+4 floats so
-// that 32 lanes reading 32 different rows hit distinct banks), lane i scores
-// key blocks i and i+32 of the chunk against the warp's query block, and the
-// list is compacted with warp ballots in ascending key-block order.
+// Two kernels.  entropy_scores_kernel is a tiled fp32 GEMM per head:
+// 64 x 64 tiles of s = Qbar Kbar^T * scale, the pooled rows staged in shared
+// memory (rows padded to D+4 floats; thread (ty, tx) owns rows ty+16i and
+// columns tx+16j, so float4 reads of neighbouring threads hit distinct banks),
+// each score accumulated over the d dimensions in order.  entropy_rows_kernel
+// gives one warp to each query block: it stages the row's scores and the
+// block cells in shared memory, reduces the scores to the entropy, maps it
+// to the radius and compacts the kept key blocks with warp ballots in
+// ascending order.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -35,15 +39,15 @@
 namespace sta {
 namespace {
 
-constexpr int kEntWarps = 8;
-constexpr int kEntThreads = kEntWarps * 32;
-constexpr int kEntChunk = 64;
+constexpr int kEntThreads = 256;
+constexpr int kScoreTile = 64;  // query x key blocks per scores CTA
+constexpr int kScoreT = kScoreTile / 16;  // rows (and columns) per thread
+constexpr int kRowWarps = 8;    // query blocks per rows CTA
 
 struct EntArgs {
-  const float* qbar;  // [heads][nb][D]
-  const float* kbar;  // [heads][nb][D]
+  const float* scores;  // [heads][nb][nb]
   int heads, nb, F, H, W, B;
-  float scale, alpha, beta;
+  float alpha, beta;
   int r_lo, r_hi, tile_h, tile_w;
   int32_t* idx;
   int32_t* cnt;
@@ -79,60 +83,100 @@ __device__ __forceinline__ float warp_max_f(float v) {
   return v;
 }
 
+// s[h][b][c] = (Qbar_b . Kbar_c) * scale for a 64 x 64 tile of (b, c).
 template <int D>
-__global__ void __launch_bounds__(kEntThreads) entropy_lists_kernel(const EntArgs a) {
-  constexpr int KS = D + 4;  // padded row stride of the staged key blocks
-  extern __shared__ float4 smem4[];
-  float* sm = reinterpret_cast<float*>(smem4);
-  float* sq = sm;                                  // [8][D]
-  float* sk = sq + kEntWarps * D;                  // [64][KS]
-  float* ss = sk + kEntChunk * KS;                 // [8][nb]
-  const int head = blockIdx.y;
-  const int qb0 = blockIdx.x * kEntWarps;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nb = a.nb;
-  const float* qh = a.qbar + static_cast<size_t>(head) * nb * D;
-  const float* kh = a.kbar + static_cast<size_t>(head) * nb * D;
-
-  for (int i = threadIdx.x; i < kEntWarps * D / 4; i += kEntThreads) {
-    const int r = (i * 4) / D;
-    const int qb = min(qb0 + r, nb - 1);
-    reinterpret_cast<float4*>(sq)[i] =
-        reinterpret_cast<const float4*>(qh + static_cast<size_t>(qb) * D)[(i * 4 - r * D) / 4];
-  }
-  for (int c0 = 0; c0 < nb; c0 += kEntChunk) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < kEntChunk * D / 4; i += kEntThreads) {
-      const int r = (i * 4) / D;
-      const int col = i * 4 - r * D;
-      const int kb = c0 + r;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (kb < nb) v = *reinterpret_cast<const float4*>(kh + static_cast<size_t>(kb) * D + col);
-      *reinterpret_cast<float4*>(sk + r * KS + col) = v;
-    }
-    __syncthreads();
-    const float4* qv = reinterpret_cast<const float4*>(sq + warp * D);
+__global__ void __launch_bounds__(kEntThreads) entropy_scores_kernel(
+    const float* __restrict__ qbar, const float* __restrict__ kbar, int nb, float scale,
+    float* __restrict__ scores) {
+  constexpr int KS = D + 4;
+  extern __shared__ float4 ssm4[];
+  float* sa = reinterpret_cast<float*>(ssm4);  // [64][KS] query rows
+  float* sb = sa + kScoreTile * KS;              // [64][KS] key rows
+  const int head = blockIdx.z;
+  const int b0 = blockIdx.y * kScoreTile, c0 = blockIdx.x * kScoreTile;
+  const float* qh = qbar + static_cast<size_t>(head) * nb * D;
+  const float* kh = kbar + static_cast<size_t>(head) * nb * D;
+  constexpr int PER = kScoreTile * D / 4 / kEntThreads;  // float4 per thread per operand
+  float4 va[PER], vb[PER];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = lane + 32 * half;
-      const float4* kv = reinterpret_cast<const float4*>(sk + r * KS);
-      float acc = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < D / 4; ++i) {
-        const float4 x = qv[i], y = kv[i];
-        acc = fmaf(x.x, y.x, acc);
-        acc = fmaf(x.y, y.y, acc);
-        acc = fmaf(x.z, y.z, acc);
-        acc = fmaf(x.w, y.w, acc);
-      }
-      if (c0 + r < nb) ss[warp * nb + c0 + r] = acc * a.scale;
-    }
+  for (int u = 0; u < PER; ++u) {
+    const int i = threadIdx.x + u * kEntThreads;
+    const int r = (i * 4) / D, col = i * 4 - r * D;
+    va[u] = b0 + r < nb ? __ldg(reinterpret_cast<const float4*>(qh + static_cast<size_t>(b0 + r) * D + col))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    vb[u] = c0 + r < nb ? __ldg(reinterpret_cast<const float4*>(kh + static_cast<size_t>(c0 + r) * D + col))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int i = threadIdx.x + u * kEntThreads;
+    const int r = (i * 4) / D, col = i * 4 - r * D;
+    *reinterpret_cast<float4*>(sa + r * KS + col) = va[u];
+    *reinterpret_cast<float4*>(sb + r * KS + col) = vb[u];
   }
   __syncthreads();
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float acc[kScoreT][kScoreT];
+#pragma unroll
+  for (int i = 0; i < kScoreT; ++i)
+#pragma unroll
+    for (int j = 0; j < kScoreT; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+  for (int k = 0; k < D; k += 4) {
+    float4 x[kScoreT], y[kScoreT];
+#pragma unroll
+    for (int i = 0; i < kScoreT; ++i)
+      x[i] = *reinterpret_cast<const float4*>(sa + (ty + 16 * i) * KS + k);
+#pragma unroll
+    for (int j = 0; j < kScoreT; ++j)
+      y[j] = *reinterpret_cast<const float4*>(sb + (tx + 16 * j) * KS + k);
+#pragma unroll
+    for (int i = 0; i < kScoreT; ++i)
+#pragma unroll
+      for (int j = 0; j < kScoreT; ++j) {
+        acc[i][j] = fmaf(x[i].x, y[j].x, acc[i][j]);
+        acc[i][j] = fmaf(x[i].y, y[j].y, acc[i][j]);
+        acc[i][j] = fmaf(x[i].z, y[j].z, acc[i][j]);
+        acc[i][j] = fmaf(x[i].w, y[j].w, acc[i][j]);
+      }
+  }
+#pragma unroll
+  for (int i = 0; i < kScoreT; ++i) {
+    const int b = b0 + ty + 16 * i;
+    if (b >= nb) continue;
+    float* out = scores + (static_cast<size_t>(head) * nb + b) * nb;
+#pragma unroll
+    for (int j = 0; j < kScoreT; ++j) {
+      const int c = c0 + tx + 16 * j;
+      if (c < nb) out[c] = acc[i][j] * scale;
+    }
+  }
+}
 
-  const int qb = qb0 + warp;
-  if (qb >= nb) return;
-  const float* s = ss + warp * nb;
+// One warp per query block: entropy of softmax over its scores, radius,
+// Chebyshev list.  Cells are packed as f << 20 | cell_h << 10 | cell_w.
+__global__ void __launch_bounds__(kRowWarps * 32) entropy_rows_kernel(const EntArgs a) {
+  extern __shared__ float rsm[];
+  const int nb = a.nb;
+  float* ss = rsm;                                             // [8][nb]
+  int* scell = reinterpret_cast<int*>(ss + kRowWarps * nb);    // [nb]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = a.F * a.H * a.W;
+  for (int b = threadIdx.x; b < nb; b += kRowWarps * 32) {
+    int cf, ch, cw;
+    block_cell(b, a.B, N, a.H, a.W, a.tile_h, a.tile_w, cf, ch, cw);
+    scell[b] = (cf << 20) | (ch << 10) | cw;
+  }
+  const int row = blockIdx.x * kRowWarps + warp;  // head*nb + qb (< 2^31: checked on the host)
+  const bool live = row < a.heads * nb;
+  float* s = ss + warp * nb;
+  if (live) {
+    const float* src = a.scores + static_cast<size_t>(row) * nb;
+    for (int c = lane; c < nb; c += 32) s[c] = __ldg(src + c);
+  }
+  __syncthreads();
+  if (!live) return;
+  const int qb = row % nb;
   float m = -INFINITY;
   for (int c = lane; c < nb; c += 32) m = fmaxf(m, s[c]);
   m = warp_max_f(m);
@@ -154,20 +198,17 @@ __global__ void __launch_bounds__(kEntThreads) entropy_lists_kernel(const EntArg
   else if (tf >= static_cast<float>(a.r_hi)) r = a.r_hi;
   else r = static_cast<int>(tf);
 
-  const int N = a.F * a.H * a.W;
-  int qf, qh_, qw;
-  block_cell(qb, a.B, N, a.H, a.W, a.tile_h, a.tile_w, qf, qh_, qw);
-  const size_t row = static_cast<size_t>(head) * nb + qb;
-  int32_t* out = a.idx + row * a.cap;
+  const int qc = scell[qb];
+  const int qf = qc >> 20, qh = (qc >> 10) & 1023, qw = qc & 1023;
+  int32_t* out = a.idx + static_cast<size_t>(row) * a.cap;
   int total = 0;
   for (int c0 = 0; c0 < nb; c0 += 32) {
     const int kb = c0 + lane;
     bool keep = false;
     if (kb < nb) {
-      int kf, kh2, kw;
-      block_cell(kb, a.B, N, a.H, a.W, a.tile_h, a.tile_w, kf, kh2, kw);
-      const int dist = max(abs(kf - qf), max(abs(kh2 - qh_), abs(kw - qw)));
-      keep = dist <= r;
+      const int kc = scell[kb];
+      const int kf = kc >> 20, kh = (kc >> 10) & 1023, kw = kc & 1023;
+      keep = max(abs(kf - qf), max(abs(kh - qh), abs(kw - qw))) <= r;
     }
     const unsigned bal = __ballot_sync(0xffffffffu, keep);
     const int pos = total + __popc(bal & ((1u << lane) - 1u));
@@ -183,49 +224,50 @@ __global__ void __launch_bounds__(kEntThreads) entropy_lists_kernel(const EntArg
   }
 }
 
-template <int D>
-size_t ent_smem(int nb) {
-  return sizeof(float) * (static_cast<size_t>(kEntWarps) * D + kEntChunk * (D + 4) +
-                          static_cast<size_t>(kEntWarps) * nb);
+size_t rows_smem(int nb) {
+  return sizeof(float) * static_cast<size_t>(kRowWarps) * nb + sizeof(int) * static_cast<size_t>(nb);
 }
 
 template <int D>
-cudaError_t launch_ent_t(const EntArgs& a, cudaStream_t s) {
-  const size_t smem = ent_smem<D>(a.nb);
-  if (smem > 227 * 1024) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(entropy_lists_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+cudaError_t launch_scores_t(const float* qbar, const float* kbar, int heads, int nb, float scale,
+                            float* scores, cudaStream_t s) {
+  const int smem = static_cast<int>(sizeof(float) * 2 * kScoreTile * (D + 4));
+  cudaError_t e = set_dyn_smem<entropy_scores_kernel<D>>(smem);
   if (e != cudaSuccess) return e;
-  dim3 g((a.nb + kEntWarps - 1) / kEntWarps, a.heads);
-  entropy_lists_kernel<D><<<g, kEntThreads, smem, s>>>(a);
+  const int nt = (nb + kScoreTile - 1) / kScoreTile;
+  entropy_scores_kernel<D><<<dim3(nt, nt, heads), kEntThreads, smem, s>>>(qbar, kbar, nb, scale,
+                                                                          scores);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 int entropy_max_blocks(int d) {
-  // key blocks whose scores fit the CTA's shared memory
-  const size_t fixed = sizeof(float) * (static_cast<size_t>(kEntWarps) * d + kEntChunk * (d + 4));
-  return static_cast<int>((227 * 1024 - fixed) / (sizeof(float) * kEntWarps));
+  (void)d;
+  // the rows kernel stages 8 score rows and the cells of all blocks
+  return static_cast<int>((227 * 1024) / (sizeof(float) * kRowWarps + sizeof(int)));
 }
 
-cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, int heads, int F, int H,
-                                 int W, int d, int B, float scale, float alpha, float beta,
-                                 int r_lo, int r_hi, int tile_h, int tile_w, int32_t* idx,
-                                 int32_t* cnt, int cap, int32_t* required_cap, float* entropy,
-                                 int32_t* radius, int32_t* dev_status, cudaStream_t s) {
+cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, float* scores, int heads,
+                                 int F, int H, int W, int d, int B, float scale, float alpha,
+                                 float beta, int r_lo, int r_hi, int tile_h, int tile_w,
+                                 int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
+                                 float* entropy, int32_t* radius, int32_t* dev_status,
+                                 cudaStream_t s) {
+  const int N = F * H * W;
+  const int nb = (N + B - 1) / B;
+  cudaError_t e = d == 128   ? launch_scores_t<128>(qbar, kbar, heads, nb, scale, scores, s)
+                  : d == 64 ? launch_scores_t<64>(qbar, kbar, heads, nb, scale, scores, s)
+                            : cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
   EntArgs a;
-  a.qbar = qbar;
-  a.kbar = kbar;
+  a.scores = scores;
   a.heads = heads;
+  a.nb = nb;
   a.F = F;
   a.H = H;
   a.W = W;
   a.B = B;
-  const int N = F * H * W;
-  a.nb = (N + B - 1) / B;
-  a.scale = scale;
   a.alpha = alpha;
   a.beta = beta;
   a.r_lo = r_lo;
@@ -239,9 +281,13 @@ cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, int heads
   a.entropy = entropy;
   a.radius = radius;
   a.dev_status = dev_status;
-  if (d == 128) return launch_ent_t<128>(a, s);
-  if (d == 64) return launch_ent_t<64>(a, s);
-  return cudaErrorInvalidValue;
+  const int smem = static_cast<int>(rows_smem(nb));
+  e = set_dyn_smem<entropy_rows_kernel>(smem);
+  if (e != cudaSuccess) return e;
+  const long long rows = static_cast<long long>(heads) * nb;
+  entropy_rows_kernel<<<static_cast<unsigned>((rows + kRowWarps - 1) / kRowWarps),
+                        kRowWarps * 32, smem, s>>>(a);
+  return cudaGetLastError();
 }
 
 }  // namespace sta

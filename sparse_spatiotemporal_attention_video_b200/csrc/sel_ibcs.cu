@@ -43,35 +43,47 @@ namespace sta {
 namespace {
 
 // ------------------------------------------------------------------ k-means
-// One CTA per (head, query block); thread r owns query row r.
-constexpr int kKmThreads = 128;
+// One CTA of 512 threads per (head, query block).  Assignment: thread
+// (g, r) = (tid / 128, tid % 128) sums the squared distance of query r over
+// dimension quarter g; the four partials are added in order g = 0..3.
+// Update: thread (g, r) sums dimension r over queries [32g, 32g+32) per
+// cluster; the four partials are added in order.  Rows of the staged block
+// have an odd stride (D+1 floats), so the 32 lanes of a warp (consecutive r)
+// hit distinct banks.
+constexpr int kKmThreads = 512;
+constexpr int kKmRows = 128;  // largest query block
 
 template <int D, int KM>
 __global__ void __launch_bounds__(kKmThreads) kmeans_kernel(
     const __nv_bfloat16* __restrict__ q, int N, int B, int nqb, int iters,
     float* __restrict__ cent, float* __restrict__ wts) {
-  constexpr int QS = D + 1;  // odd row stride: lanes of one column hit distinct banks
+  constexpr int QS = D + 1;
+  constexpr int DQ = D / 4;  // dimensions per quarter
   extern __shared__ float km_smem[];
-  float* sq = km_smem;                  // [B][QS]
-  float* sc = sq + kKmThreads * QS;     // [KM][D]
-  int* sassign = reinterpret_cast<int*>(sc + KM * D);  // [B]
+  float* sq = km_smem;                       // [128][QS]
+  float* sc = sq + kKmRows * QS;             // [KM][D]
+  float* part = sc + KM * D;                 // [4][128][KM] distances / [4][KM][D] sums
+  int* sassign = reinterpret_cast<int*>(part + 4 * kKmRows * KM);  // [128]
+  int* pcount = sassign + kKmRows;           // [4][KM]
   __shared__ int scount[KM];
   const int row = blockIdx.x;  // head * nqb + qb
   const int head = row / nqb;
   const int qb = row - head * nqb;
   const int q0 = qb * B;
   const int nb = min(B, N - q0);
+  const int g = threadIdx.x / kKmRows;
+  const int r = threadIdx.x - g * kKmRows;
   const __nv_bfloat16* qh = q + (static_cast<size_t>(head) * N + q0) * D;
   // stage the block as fp32 (rows >= nb are never read)
   for (int i = threadIdx.x; i < nb * D / 8; i += kKmThreads) {
-    const int r = (i * 8) / D;
-    const int c = i * 8 - r * D;
+    const int rr = (i * 8) / D;
+    const int c = i * 8 - rr * D;
     const uint4 v = __ldcs(reinterpret_cast<const uint4*>(qh) + i);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
-      sq[r * QS + c + 2 * t] = __uint_as_float(w[t] << 16);
-      sq[r * QS + c + 2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
+      sq[rr * QS + c + 2 * t] = __uint_as_float(w[t] << 16);
+      sq[rr * QS + c + 2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
     }
   }
   __syncthreads();
@@ -80,14 +92,15 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_kernel(
     sc[i] = sq[((c * nb) / KM) * QS + col];
   }
   __syncthreads();
-  const int r = threadIdx.x;
   for (int it = 0; it < iters; ++it) {
-    // assignment
+    // assignment: partial squared distances over one quarter of the dims
     if (r < nb) {
       float d2[KM];
 #pragma unroll
       for (int c = 0; c < KM; ++c) d2[c] = 0.f;
-      for (int col = 0; col < D; ++col) {
+#pragma unroll 8
+      for (int i = 0; i < DQ; ++i) {
+        const int col = g * DQ + i;
         const float x = sq[r * QS + col];
 #pragma unroll
         for (int c = 0; c < KM; ++c) {
@@ -95,14 +108,27 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_kernel(
           d2[c] = fmaf(t, t, d2[c]);
         }
       }
-      int best = 0;
 #pragma unroll
-      for (int c = 1; c < KM; ++c)
-        if (d2[c] < d2[best]) best = c;
+      for (int c = 0; c < KM; ++c) part[(g * kKmRows + r) * KM + c] = d2[c];
+    }
+    __syncthreads();
+    if (g == 0 && r < nb) {
+      int best = 0;
+      float bd = 0.f;
+#pragma unroll
+      for (int c = 0; c < KM; ++c) {
+        float d = part[r * KM + c];
+#pragma unroll
+        for (int gg = 1; gg < 4; ++gg) d += part[(gg * kKmRows + r) * KM + c];
+        if (c == 0 || d < bd) {
+          bd = d;
+          best = c;
+        }
+      }
       sassign[r] = best;
     }
     __syncthreads();
-    // update: thread = column (D <= 128 = threads)
+    // update: partial member sums of dimension r over one quarter of the queries
     if (r < D) {
       float acc[KM];
       int n[KM];
@@ -111,23 +137,35 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_kernel(
         acc[c] = 0.f;
         n[c] = 0;
       }
-      for (int t = 0; t < nb; ++t) {
-        const int a = sassign[t];
+      const int t1 = min(nb, (g + 1) * (kKmRows / 4));
+      for (int t = g * (kKmRows / 4); t < t1; ++t) {
+        const int as = sassign[t];
         const float x = sq[t * QS + r];
 #pragma unroll
         for (int c = 0; c < KM; ++c) {
-          if (a == c) {
+          if (as == c) {
             acc[c] += x;
             ++n[c];
           }
         }
       }
 #pragma unroll
-      for (int c = 0; c < KM; ++c)
-        if (n[c] > 0) sc[c * D + r] = acc[c] / static_cast<float>(n[c]);
+      for (int c = 0; c < KM; ++c) part[(g * KM + c) * D + r] = acc[c];
       if (r == 0) {
 #pragma unroll
-        for (int c = 0; c < KM; ++c) scount[c] = n[c];
+        for (int c = 0; c < KM; ++c) pcount[g * KM + c] = n[c];
+      }
+    }
+    __syncthreads();
+    if (g == 0 && r < D) {
+#pragma unroll
+      for (int c = 0; c < KM; ++c) {
+        const int n = pcount[c] + pcount[KM + c] + pcount[2 * KM + c] + pcount[3 * KM + c];
+        float acc = part[c * D + r];
+#pragma unroll
+        for (int gg = 1; gg < 4; ++gg) acc += part[(gg * KM + c) * D + r];
+        if (n > 0) sc[c * D + r] = acc / static_cast<float>(n);
+        if (r == 0) scount[c] = n;
       }
     }
     __syncthreads();
@@ -147,10 +185,11 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_kernel(
 // transposed (As[k][row]); sub-block-mean chunks are double-buffered through
 // registers (Bs[k][j]).  Thread (ty, tx) owns rows ty*8..ty*8+7 (8/KM whole
 // query blocks) and columns tx*4..tx*4+3 and 64+tx*4..64+tx*4+3 (two float4
-// reads per k that fall on distinct banks).  Sweep 1 over all sub-blocks
-// keeps an online max and an fp64 sum of exp per row; the 16 threads of a
-// row group then merge them.  Sweep 2 recomputes the scores and writes
-// p_j = sum_c (w_c / Z_c) exp(z_cj - M_c) for each query block.
+// reads per k that fall on distinct banks).  One sweep over all sub-blocks
+// stores the scores z_cj and keeps an online max and an fp64 sum of exp per
+// row; the 16 threads of a row group then merge them into (w_c / Z_c, M_c).
+// Storing z (4 B per score, written and read once) is cheaper than a second
+// sweep of the GEMM; sip_sample_kernel forms p from it.
 constexpr int kImpThreads = 256;
 constexpr int kImpRows = 128;
 constexpr int kImpCols = 128;
@@ -168,9 +207,8 @@ template <int D, int KM>
 __global__ void __launch_bounds__(kImpThreads, 1) importance_kernel(
     const float* __restrict__ cent, const float* __restrict__ wts,
     const float* __restrict__ kbar, int nqb, int n_sub, int N, int U, float scale,
-    float* __restrict__ p) {
+    float* __restrict__ zout, float* __restrict__ stats) {
   static_assert(8 % KM == 0, "centroids per query block must divide 8");
-  constexpr int QPT = 8 / KM;  // query blocks per thread
   constexpr int NCH = D / kImpKc;
   extern __shared__ float4 imp_smem4[];
   float* As = reinterpret_cast<float*>(imp_smem4);     // [D][kImpRows + pad]
@@ -273,6 +311,18 @@ __global__ void __launch_bounds__(kImpThreads, 1) importance_kernel(
   for (int j0 = 0; j0 < n_sub; j0 += kImpCols) {
     float z[8][8];
     tile_scores(j0, z);
+    // keep the scores: p is formed from them once the normalisers are known
+#pragma unroll
+    for (int x = 0; x < 8; ++x) {
+      const int r = row0 + ty * 8 + x;
+      if (r >= n_rows) continue;
+      float* zr = zout + (static_cast<size_t>(head) * n_rows + r) * n_sub + j0;
+#pragma unroll
+      for (int y = 0; y < 8; ++y) {
+        const int c = y < 4 ? tx * 4 + y : 64 + tx * 4 + (y - 4);
+        if (j0 + c < n_sub) zr[c] = z[x][y];
+      }
+    }
 #pragma unroll
     for (int x = 0; x < 8; ++x) {
       float t = z[x][0];
@@ -304,53 +354,18 @@ __global__ void __launch_bounds__(kImpThreads, 1) importance_kernel(
       s[x] = acc;
     }
   }
-  // coefficient w_c / Z_c per row
-  float coef[8];
+  // per centroid row: coefficient w_c / Z_c and the maximum M_c
+  if (tx == 0) {
 #pragma unroll
-  for (int x = 0; x < 8; ++x) {
-    const int r = row0 + ty * 8 + x;
-    coef[x] = 0.f;
-    if (r < n_rows && s[x] > 0.0)
-      coef[x] = static_cast<float>(static_cast<double>(__ldg(wts + static_cast<size_t>(head) * n_rows + r)) / s[x]);
-  }
-
-  // ---- sweep 2: p for each query block of this thread
-  for (int j0 = 0; j0 < n_sub; j0 += kImpCols) {
-    float z[8][8];
-    tile_scores(j0, z);
-#pragma unroll
-    for (int qq = 0; qq < QPT; ++qq) {
-      const int r = row0 + ty * 8 + qq * KM;
-      const int qb = r / KM;
-      float out[8];
-#pragma unroll
-      for (int y = 0; y < 8; ++y) {
-        float acc = 0.f;
-#pragma unroll
-        for (int c = 0; c < KM; ++c) {
-          const int x = qq * KM + c;
-          if (coef[x] != 0.f) acc = fmaf(coef[x], expf(z[x][y] - m[x]), acc);
-        }
-        out[y] = acc;
-      }
-      if (r < n_rows) {
-        float* pr = p + (static_cast<size_t>(head) * nqb + qb) * n_sub + j0;
-        const int c0 = tx * 4, c1 = 64 + tx * 4;
-        if (j0 + c0 + 3 < n_sub && ((n_sub & 3) == 0)) {
-          *reinterpret_cast<float4*>(pr + c0) = make_float4(out[0], out[1], out[2], out[3]);
-        } else {
-#pragma unroll
-          for (int y = 0; y < 4; ++y)
-            if (j0 + c0 + y < n_sub) pr[c0 + y] = out[y];
-        }
-        if (j0 + c1 + 3 < n_sub && ((n_sub & 3) == 0)) {
-          *reinterpret_cast<float4*>(pr + c1) = make_float4(out[4], out[5], out[6], out[7]);
-        } else {
-#pragma unroll
-          for (int y = 0; y < 4; ++y)
-            if (j0 + c1 + y < n_sub) pr[c1 + y] = out[4 + y];
-        }
-      }
+    for (int x = 0; x < 8; ++x) {
+      const int r = row0 + ty * 8 + x;
+      if (r >= n_rows) continue;
+      float coef = 0.f;
+      if (s[x] > 0.0)
+        coef = static_cast<float>(
+            static_cast<double>(__ldg(wts + static_cast<size_t>(head) * n_rows + r)) / s[x]);
+      float2* st = reinterpret_cast<float2*>(stats) + static_cast<size_t>(head) * n_rows + r;
+      *st = make_float2(coef, m[x]);
     }
   }
 }
@@ -411,20 +426,46 @@ __device__ __forceinline__ int block_sum_i(int v, int* red, int& excl) {
   return tot;
 }
 
+template <int KM>
 __global__ void __launch_bounds__(kSipThreads) sip_sample_kernel(
-    const float* __restrict__ p, int nqb, int n_sub, int m, uint32_t seed_lo, uint32_t seed_hi,
-    int32_t* __restrict__ idx, float* __restrict__ logw, int32_t* __restrict__ cnt, int cap,
-    int32_t* required_cap, int32_t* dev_status) {
+    const float* __restrict__ z, const float* __restrict__ stats, int n_sub, int m,
+    uint32_t seed_lo, uint32_t seed_hi, int32_t* __restrict__ idx, float* __restrict__ logw,
+    int32_t* __restrict__ cnt, int cap, int32_t* required_cap, int32_t* dev_status) {
   extern __shared__ float sip_smem[];
   float* sp = sip_smem;                                    // [n_sub]
   uint8_t* capped = reinterpret_cast<uint8_t*>(sp + n_sub);  // [n_sub]
   __shared__ double redd[kSipWarps];
   __shared__ int redi[kSipWarps];
+  __shared__ float2 cs[KM];
   const int row = blockIdx.x;  // head * nqb + qb
-  const float* pr = p + static_cast<size_t>(row) * n_sub;
-  for (int j = threadIdx.x; j < n_sub; j += kSipThreads) {
-    sp[j] = pr[j];
-    capped[j] = 0;
+  if (threadIdx.x < KM)
+    cs[threadIdx.x] = reinterpret_cast<const float2*>(stats)[static_cast<size_t>(row) * KM + threadIdx.x];
+  __syncthreads();
+  // p_j = sum_c (w_c / Z_c) exp(z_cj - M_c), centroids in order; the scores
+  // of four j per thread are loaded before any is used
+  const float* zr = z + static_cast<size_t>(row) * KM * n_sub;
+  for (int j0 = threadIdx.x; j0 < n_sub; j0 += 4 * kSipThreads) {
+    float zv[4][KM];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * kSipThreads;
+#pragma unroll
+      for (int c = 0; c < KM; ++c)
+        zv[u][c] = j < n_sub ? __ldcs(zr + static_cast<size_t>(c) * n_sub + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * kSipThreads;
+      if (j >= n_sub) break;
+      float acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < KM; ++c) {
+        const float2 cm = cs[c];
+        if (cm.x != 0.f) acc = fmaf(cm.x, expf(zv[u][c] - cm.y), acc);
+      }
+      sp[j] = acc;
+      capped[j] = 0;
+    }
   }
   __syncthreads();
   // water filling
@@ -501,35 +542,32 @@ __global__ void __launch_bounds__(kSipThreads) sip_sample_kernel(
 
 template <int D, int KM>
 cudaError_t launch_ibcs_t(const __nv_bfloat16* q, const float* kbar, float* cent, float* wts,
-                          float* p, int heads, int N, int B, int U, int iters, int m,
+                          float* z, float* stats, int heads, int N, int B, int U, int iters, int m,
                           uint64_t seed, float scale, int32_t* idx, float* logw, int32_t* cnt,
                           int cap, int32_t* required_cap, int32_t* dev_status, cudaStream_t s) {
   const int nqb = (N + B - 1) / B;
   const int n_sub = (N + U - 1) / U;
-  const size_t km_smem = sizeof(float) * (static_cast<size_t>(kKmThreads) * (D + 1) + KM * D) +
-                         sizeof(int) * kKmThreads;
-  cudaError_t e = cudaFuncSetAttribute(kmeans_kernel<D, KM>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(km_smem));
+  const size_t km_smem =
+      sizeof(float) * (static_cast<size_t>(kKmRows) * (D + 1) + KM * D + 4 * kKmRows * KM) +
+      sizeof(int) * (kKmRows + 4 * KM);
+  cudaError_t e = set_dyn_smem<kmeans_kernel<D, KM>>(static_cast<int>(km_smem));
   if (e != cudaSuccess) return e;
   kmeans_kernel<D, KM><<<heads * nqb, kKmThreads, km_smem, s>>>(q, N, B, nqb, iters, cent, wts);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const size_t imp_smem = imp_smem_bytes<D>();
-  e = cudaFuncSetAttribute(importance_kernel<D, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(imp_smem));
+  e = set_dyn_smem<importance_kernel<D, KM>>(static_cast<int>(imp_smem));
   if (e != cudaSuccess) return e;
   dim3 gi((nqb * KM + kImpRows - 1) / kImpRows, heads);
   importance_kernel<D, KM><<<gi, kImpThreads, imp_smem, s>>>(cent, wts, kbar, nqb, n_sub, N, U,
-                                                             scale, p);
+                                                             scale, z, stats);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const size_t sip_smem = static_cast<size_t>(n_sub) * (sizeof(float) + 1);
-  e = cudaFuncSetAttribute(sip_sample_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(sip_smem));
+  e = set_dyn_smem<sip_sample_kernel<KM>>(static_cast<int>(sip_smem));
   if (e != cudaSuccess) return e;
-  sip_sample_kernel<<<heads * nqb, kSipThreads, sip_smem, s>>>(
-      p, nqb, n_sub, m, static_cast<uint32_t>(seed & 0xffffffffu), static_cast<uint32_t>(seed >> 32),
+  sip_sample_kernel<KM><<<heads * nqb, kSipThreads, sip_smem, s>>>(
+      z, stats, n_sub, m, static_cast<uint32_t>(seed & 0xffffffffu), static_cast<uint32_t>(seed >> 32),
       idx, logw, cnt, cap, required_cap, dev_status);
   return cudaGetLastError();
 }
@@ -539,13 +577,13 @@ cudaError_t launch_ibcs_t(const __nv_bfloat16* q, const float* kbar, float* cent
 int ibcs_max_subblocks() { return static_cast<int>((200 * 1024) / (sizeof(float) + 1)); }
 
 cudaError_t launch_ibcs_sip(const __nv_bfloat16* q, const float* kbar, float* cent, float* wts,
-                            float* p, int heads, int N, int d, int B, int U, int km_k, int iters,
+                            float* z, float* stats, int heads, int N, int d, int B, int U, int km_k, int iters,
                             int m, uint64_t seed, float scale, int32_t* idx, float* logw,
                             int32_t* cnt, int cap, int32_t* required_cap, int32_t* dev_status,
                             cudaStream_t s) {
 #define STA_IBCS_CASE(DD, KK)                                                                   \
   if (d == DD && km_k == KK)                                                                    \
-    return launch_ibcs_t<DD, KK>(q, kbar, cent, wts, p, heads, N, B, U, iters, m, seed, scale, \
+    return launch_ibcs_t<DD, KK>(q, kbar, cent, wts, z, stats, heads, N, B, U, iters, m, seed, scale, \
                                  idx, logw, cnt, cap, required_cap, dev_status, s);
   STA_IBCS_CASE(128, 4)
   STA_IBCS_CASE(128, 2)

@@ -137,7 +137,7 @@ sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16*
 
 // Workspace carve-up of the content selectors (256-byte aligned segments).
 struct SelWorkspace {
-  size_t qbar = 0, kbar = 0, cent = 0, wts = 0, p = 0, total = 0;
+  size_t qbar = 0, kbar = 0, scores = 0, cent = 0, wts = 0, z = 0, stats = 0, total = 0;
 };
 
 SelWorkspace sel_workspace(const sta_problem* p, const sta_selector_params* sel) {
@@ -157,12 +157,14 @@ SelWorkspace sel_workspace(const sta_problem* p, const sta_selector_params* sel)
   if (sel->kind == STA_SEL_ENTROPY) {
     w.qbar = take(h * nqb * d * 4);
     w.kbar = take(h * nku * d * 4);
+    w.scores = take(h * nqb * nku * 4);
   } else if (sel->kind == STA_SEL_IBCS_SIP) {
     const size_t km = sel->km_k > 0 ? static_cast<size_t>(sel->km_k) : 1;
     w.kbar = take(h * nku * d * 4);
     w.cent = take(h * nqb * km * d * 4);
     w.wts = take(h * nqb * km * 4);
-    w.p = take(h * nqb * nku * 4);
+    w.z = take(h * nqb * km * nku * 4);
+    w.stats = take(h * nqb * km * 8);
   }
   w.total = off;
   return w;
@@ -257,6 +259,10 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       const int N = prob->F * prob->H * prob->W;
       const int nb = (N + sel->block_q - 1) / sel->block_q;
       if (nb > entropy_max_blocks(prob->d)) return STA_ERR_UNSUPPORTED;
+      // block cells are packed in 11 + 10 + 10 bits
+      if (prob->F > 2047 || (prob->H - 1) / sel->ent_tile_h > 1023 ||
+          (prob->W - 1) / sel->ent_tile_w > 1023)
+        return STA_ERR_UNSUPPORTED;
       const SelWorkspace w = sel_workspace(prob, sel);
       if (!workspace || workspace_bytes < w.total) return STA_ERR_WORKSPACE;
       uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -268,11 +274,13 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
                              static_cast<const __nv_bfloat16*>(k), qbar, kbar, prob->heads, N,
                              prob->d, sel->block_q, s)))
         return STA_ERR_CUDA;
-      if (failed(launch_entropy_lists(qbar, kbar, prob->heads, prob->F, prob->H, prob->W, prob->d,
-                               sel->block_q, scale, sel->ent_alpha, sel->ent_beta, sel->ent_r_lo,
-                               sel->ent_r_hi, sel->ent_tile_h, sel->ent_tile_w, out->idx,
-                               out->cnt, out->cap, out->required_cap, out->entropy, out->radius,
-                               dev_status, s)))
+      if (failed(launch_entropy_lists(qbar, kbar, reinterpret_cast<float*>(ws + w.scores),
+                                      prob->heads, prob->F, prob->H, prob->W, prob->d,
+                                      sel->block_q, scale, sel->ent_alpha, sel->ent_beta,
+                                      sel->ent_r_lo, sel->ent_r_hi, sel->ent_tile_h,
+                                      sel->ent_tile_w, out->idx, out->cnt, out->cap,
+                                      out->required_cap, out->entropy, out->radius, dev_status,
+                                      s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }
@@ -308,14 +316,15 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       float* kbar = reinterpret_cast<float*>(ws + w.kbar);
       float* cent = reinterpret_cast<float*>(ws + w.cent);
       float* wts = reinterpret_cast<float*>(ws + w.wts);
-      float* pbuf = reinterpret_cast<float*>(ws + w.p);
+      float* zbuf = reinterpret_cast<float*>(ws + w.z);
+      float* sbuf = reinterpret_cast<float*>(ws + w.stats);
       out->head_shared = 0;
       const int m = fraction_count(sel->sample_frac, n_sub, 1);
       const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
       if (failed(launch_block_means(static_cast<const __nv_bfloat16*>(k), nullptr, kbar, nullptr,
                              prob->heads, N, prob->d, sel->kv_unit, s)))
         return STA_ERR_CUDA;
-      if (failed(launch_ibcs_sip(static_cast<const __nv_bfloat16*>(q), kbar, cent, wts, pbuf,
+      if (failed(launch_ibcs_sip(static_cast<const __nv_bfloat16*>(q), kbar, cent, wts, zbuf, sbuf,
                           prob->heads, N, prob->d, sel->block_q, sel->kv_unit, sel->km_k,
                           sel->km_iters, m, sel->seed, scale, out->idx, out->logw, out->cnt,
                           out->cap, out->required_cap, dev_status, s)))
