@@ -280,28 +280,40 @@ __device__ __forceinline__ void mask_half(float (&x)[64], const HalfInfo<UNIT>& 
     for (int c = 0; c < 64; ++c) x[c] += hi.braw[c / W];
   }
   if (window) {
-    // key coordinates advance column by column; they are recomputed from the
-    // slot's first token at every slot boundary
+    // Per slot: when the slot's W keys lie in one grid row (same f and h),
+    // the window is one column interval [lo, hi) of the slot; otherwise the
+    // key coordinates are walked column by column.
     const int S = a.H * a.W;
-    int f = 0, h = 0, w = 0;
 #pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      if ((c % W) == 0) {
-        const int t0 = hi.tok0[c / W];
-        f = t0 / S;
-        const int rem = t0 - f * S;
-        h = rem / a.W;
-        w = rem - h * a.W;
-      }
-      const int df = f - fq, dh = h - hq, dw = w - wq;
-      const bool in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
-                      (dh < a.win_h) && (dw >= -a.win_w) && (dw < a.win_w);
-      if (!in) x[c] = -INFINITY;
-      if (++w == a.W) {
-        w = 0;
-        if (++h == a.H) {
-          h = 0;
-          ++f;
+    for (int sl = 0; sl < HalfInfo<UNIT>::SLOTS; ++sl) {
+      const int t0 = hi.tok0[sl];
+      int f = t0 / S;
+      const int rem = t0 - f * S;
+      int h = rem / a.W;
+      int w = rem - h * a.W;
+      if (w + W <= a.W) {
+        const int df = f - fq, dh = h - hq;
+        const bool row_in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
+                            (dh < a.win_h);
+        const int lo = row_in ? wq - a.win_w - w : W;
+        const int hi_c = row_in ? wq + a.win_w - w : 0;
+#pragma unroll
+        for (int c = 0; c < W; ++c)
+          if (c < lo || c >= hi_c) x[sl * W + c] = -INFINITY;
+      } else {
+#pragma unroll
+        for (int c = 0; c < W; ++c) {
+          const int df = f - fq, dh = h - hq, dw = w - wq;
+          const bool in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
+                          (dh < a.win_h) && (dw >= -a.win_w) && (dw < a.win_w);
+          if (!in) x[sl * W + c] = -INFINITY;
+          if (++w == a.W) {
+            w = 0;
+            if (++h == a.H) {
+              h = 0;
+              ++f;
+            }
+          }
         }
       }
     }
