@@ -264,8 +264,10 @@ __device__ __forceinline__ void half_info_from_raw(const AttnArgs& a, const Item
   }
 }
 
-// Masks (partial units, key tokens past N), log-weights and the local window
-// on one group's 64 logit columns.
+// Masks (partial units, key tokens past N) and the local window on one
+// group's 64 logit columns.  Log-weights are not added here: they are
+// constant per slot, so the caller folds them into the per-slot maxima and
+// into the exponent's offset.
 template <int UNIT>
 __device__ __forceinline__ void mask_half(float (&x)[64], const HalfInfo<UNIT>& hi, bool window,
                                           const AttnArgs& a, int fq, int hq, int wq) {
@@ -274,10 +276,6 @@ __device__ __forceinline__ void mask_half(float (&x)[64], const HalfInfo<UNIT>& 
 #pragma unroll
     for (int c = 0; c < 64; ++c)
       if ((c % W) >= hi.lim[c / W]) x[c] = -INFINITY;
-  }
-  if (hi.bias) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) x[c] += hi.braw[c / W];
   }
   if (window) {
     // Per slot: when the slot's W keys lie in one grid row (same f and h),
@@ -333,20 +331,23 @@ struct SoftmaxShared {
 
 __device__ __forceinline__ float nan_flag() { return __int_as_float(0x7fc00000); }
 
-// Exponentials of one 64-column half: p = 2^(x*scale_log2 - m), packed to
-// bf16 pairs; returns the sum of the rounded values.  The scale-and-shift and
-// the running sums use the paired fp32 instructions (two lanes of work per
-// instruction).
-__device__ __forceinline__ float exp_pack_half(const float (&x)[64], float scale_log2, float m,
-                                               bool simple, uint32_t (&pk)[32]) {
+// Exponentials of one 64-column half: p = 2^(x*scale_log2 + off[s]) with the
+// offset off[s] = log-weight - m of the column's slot (W columns each), packed
+// to bf16 pairs; returns the sum of the rounded values.  The scale-and-shift
+// and the running sums use the paired fp32 instructions (two lanes of work
+// per instruction).
+template <int W>
+__device__ __forceinline__ float exp_pack_half(const float (&x)[64], float scale_log2,
+                                               const float (&off)[64 / W], bool simple,
+                                               uint32_t (&pk)[32]) {
   const float2 sl = make_float2(scale_log2, scale_log2);
-  const float2 nm = make_float2(-m, -m);
   float2 acc[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int c = 0; c < 64; c += 2) {
-    const float2 arg = __ffma2_rn(make_float2(x[c], x[c + 1]), sl, nm);
+    const float o = off[c / W];
+    const float2 arg = __ffma2_rn(make_float2(x[c], x[c + 1]), sl, make_float2(o, o));
     float p0, p1;
 #if STA_POLY_EVERY > 0
     // one pair in every STA_POLY_EVERY on the FMA pipe (finite arguments only)
@@ -371,14 +372,23 @@ __device__ __forceinline__ float exp_pack_half(const float (&x)[64], float scale
   return t.x + t.y;
 }
 
-__device__ __forceinline__ float max64(const float (&x)[64]) {
-  float mv[8];
+// Largest logit of each W-column slot.
+template <int W>
+__device__ __forceinline__ void slot_max(const float (&x)[64], float (&ms)[64 / W]) {
+  constexpr int A = W >= 32 ? 8 : 4;  // independent max chains per slot
 #pragma unroll
-  for (int j = 0; j < 8; ++j) mv[j] = x[j];
+  for (int s = 0; s < 64 / W; ++s) {
+    float mv[A];
 #pragma unroll
-  for (int c = 8; c < 64; ++c) mv[c & 7] = fmaxf(mv[c & 7], x[c]);
-  return fmaxf(fmaxf(fmaxf(mv[0], mv[1]), fmaxf(mv[2], mv[3])),
-               fmaxf(fmaxf(mv[4], mv[5]), fmaxf(mv[6], mv[7])));
+    for (int j = 0; j < A; ++j) mv[j] = x[s * W + j];
+#pragma unroll
+    for (int c = A; c < W; ++c) mv[c % A] = fmaxf(mv[c % A], x[s * W + c]);
+#pragma unroll
+    for (int j = A / 2; j > 0; j /= 2)
+#pragma unroll
+      for (int i = 0; i < j; ++i) mv[i] = fmaxf(mv[i], mv[i + j]);
+    ms[s] = mv[0];
+  }
 }
 
 // Loads 64 consecutive TMEM columns starting at taddr (this thread's lane).
@@ -480,7 +490,17 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         if (dense_like) mask_half<kTileK>(x, td, false, a, 0, 0, 0);
         else mask_half<UNIT>(x, ti, window, a, fq, hq, wq);
       }
-      const float m_tile = max64(x) * scale_log2;  // -inf if all masked
+      // per-slot log-weights (raw logit units), 0 without weights
+      constexpr int SW = HalfInfo<UNIT>::W, NS = HalfInfo<UNIT>::SLOTS;
+      float bias[NS];
+#pragma unroll
+      for (int q = 0; q < NS; ++q) bias[q] = (!dense_like && ti.bias) ? ti.braw[q] : 0.f;
+      float ms[NS];
+      slot_max<SW>(x, ms);
+      float mraw = ms[0] + bias[0];
+#pragma unroll
+      for (int q = 1; q < NS; ++q) mraw = fmaxf(mraw, ms[q] + bias[q]);
+      const float m_tile = mraw * scale_log2;  // -inf if all masked
       const float m_new = fmaxf(m_run, m_tile);
       const bool need = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
       if (__any_sync(0xffffffffu, need)) {
@@ -514,7 +534,10 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       // P of this group's 64 keys, packed over the first 32 of its (already
       // read) logit columns
       uint32_t pk[32];
-      l_run += exp_pack_half(x, scale_log2, m_use, simple, pk);
+      float off[NS];
+#pragma unroll
+      for (int q = 0; q < NS; ++q) off[q] = fmaf(bias[q], scale_log2, -m_use);
+      l_run += exp_pack_half<SW>(x, scale_log2, off, simple, pk);
       tmem_st32(tS + J * 64, pk);
       tmem_wait_st();
       tc_fence_before();
