@@ -255,6 +255,19 @@ const char* sta_dev_status_string(int32_t bits);
  */
 const char* sta_last_cuda_error(void);
 
+/*
+ * Self-test of the bounded waits that every kernel of this library uses (no
+ * counterpart on the pages; it supports failure detection).  One CTA waits on
+ * a barrier phase that nothing completes, with a limit of limit_ns
+ * nanoseconds of GPU global time (0 < limit_ns <= 2e9).  When the limit runs
+ * out the kernel gives up, ORs STA_DEV_TIMEOUT into *dev_status, writes 0 to
+ * *waited_ok (1 would mean the wait completed) and returns; it never traps,
+ * so the context stays usable.  dev_status and waited_ok: device int32.
+ * Errors: STA_ERR_ARG, STA_ERR_CUDA.
+ */
+sta_status sta_selftest_bounded_wait(uint64_t limit_ns, int32_t* dev_status, int32_t* waited_ok,
+                                     sta_stream_t stream);
+
 /* Library version (major*10000 + minor*100 + patch). */
 int sta_version(void);
 

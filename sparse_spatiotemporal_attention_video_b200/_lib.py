@@ -87,6 +87,8 @@ SIGNATURES = {
     "sta_dev_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "sta_version": (ctypes.c_int, []),
     "sta_last_cuda_error": (ctypes.c_char_p, []),
+    "sta_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_void_p]),
 }
 
 _lib = None

@@ -121,4 +121,8 @@ cudaError_t launch_ibcs_sip(const __nv_bfloat16* q, const float* kbar, float* ce
                             int32_t* cnt, int cap, int32_t* required_cap, int32_t* dev_status,
                             cudaStream_t s);
 
+// Self-test of the bounded wait (selftest.cu).
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* dev_status,
+                                         int32_t* waited_ok, cudaStream_t s);
+
 }  // namespace sta

@@ -1,0 +1,38 @@
+// selftest.cu -- exercises the bounded wait every kernel of this library uses
+// (mbar_wait): one CTA waits on an mbarrier phase that nothing completes, with
+// a caller-chosen limit, and must give up, raise STA_DEV_TIMEOUT and return.
+// The GPU context stays usable afterwards; no trap, no fault.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace sta {
+namespace {
+
+__global__ void bounded_wait_kernel(uint64_t limit_ns, int32_t* dev_status, int32_t* waited_ok) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);  // one arrival expected; none is ever made
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile int* ab = &abort_flag;
+    const bool ok = mbar_wait(&bar, 0, ab, limit_ns);
+    *waited_ok = ok ? 1 : 0;
+    if (!ok) raise_status(dev_status, STA_DEV_TIMEOUT);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* dev_status,
+                                         int32_t* waited_ok, cudaStream_t s) {
+  bounded_wait_kernel<<<1, 32, 0, s>>>(limit_ns, dev_status, waited_ok);
+  return cudaGetLastError();
+}
+
+}  // namespace sta

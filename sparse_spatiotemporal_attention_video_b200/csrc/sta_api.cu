@@ -185,6 +185,16 @@ extern "C" {
 
 int sta_version(void) { return kVersion; }
 
+sta_status sta_selftest_bounded_wait(uint64_t limit_ns, int32_t* dev_status, int32_t* waited_ok,
+                                     sta_stream_t stream) {
+  if (!dev_status || !waited_ok) return STA_ERR_ARG;
+  if (limit_ns == 0 || limit_ns > kWaitLimitNs) return STA_ERR_ARG;
+  if (failed(launch_bounded_wait_selftest(limit_ns, dev_status, waited_ok,
+                                          reinterpret_cast<cudaStream_t>(stream))))
+    return STA_ERR_CUDA;
+  return STA_OK;
+}
+
 const char* sta_last_cuda_error(void) {
   return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
 }

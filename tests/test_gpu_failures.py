@@ -1,0 +1,90 @@
+"""Failure detection without a GPU fault: a bounded wait that runs out
+reports STA_DEV_TIMEOUT and leaves the context usable; list rows longer than
+their capacity are truncated, flagged and their true length reported; an
+out-of-range list entry is skipped and flagged."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import radial
+from oracle.pipeline import block_sparse_rows
+from synthetic import make_qkv, workload
+from tests._util import assert_close_attn
+
+pytestmark = pytest.mark.gpu
+
+
+def _mods():
+    from sparse_spatiotemporal_attention_video_b200 import _lib, api, session
+    return _lib, api, session
+
+
+def test_bounded_wait_times_out_and_context_survives(cuda_ok):
+    _lib, api, session = _mods()
+    lib = _lib.load()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    waited = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    code = lib.sta_selftest_bounded_wait(50_000_000, st.data_ptr(), waited.data_ptr(),
+                                         torch.cuda.current_stream().cuda_stream)
+    assert code == _lib.STA_OK
+    torch.cuda.synchronize()
+    assert int(waited.item()) == 0
+    assert int(st.item()) & _lib.STA_DEV_TIMEOUT
+    # the context is still usable: a normal dense call gives the right result
+    w = workload("wan_radial", heads=1, F=2, H=8, W=16)
+    q, k, v = make_qkv(w)
+    o = torch.empty(q.shape, dtype=q.dtype, device="cuda")
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    api.sta_dense_attn_fwd(session.problem(w), q.cuda(), k.cuda(), v.cuda(), 0.0, o,
+                           dev_status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 0
+    ref = np.concatenate([block_sparse_rows(q[0], k[0], v[0], b, list(range(2)), 128, 128)
+                          for b in range(2)])
+    assert_close_attn(o[0].float().cpu().numpy(), ref, "dense after timeout")
+
+
+def test_capacity_overflow_truncates_and_reports(cuda_ok):
+    _lib, api, session = _mods()
+    w = workload("wan_radial")
+    ref = radial.block_lists(w["F"], w["H"], w["W"], w["block_q"], w["radial"])
+    need = max(len(r) for r in ref)
+    cap = need // 3
+    L = session.Lists(w, cap=cap)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    api.sta_build_blocks(session.problem(w), session.selector(w), None, None, L.struct,
+                         dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & _lib.STA_DEV_CAPACITY
+    assert int(L.required_cap.item()) == need
+    got = L.host_rows()
+    for qb, r in enumerate(ref):
+        assert got[qb] == list(r)[:cap]
+
+
+def test_out_of_range_entry_is_skipped_and_flagged(cuda_ok):
+    _lib, api, session = _mods()
+    from sparse_spatiotemporal_attention_video_b200._lib import AttnParams, BlockLists
+    w = workload("wan_radial", heads=1, F=3, H=10, W=13, kv_unit=32)   # N = 390
+    q, k, v = make_qkv(w)
+    n_units = (w["N"] + 31) // 32
+    idx = np.array([[0, 3, n_units + 5, 7], [1, 2, 4, 9], [5, -1, 6, 10], [11, 12, 0, 0]],
+                   np.int32)
+    cnt = np.array([4, 4, 4, 2], np.int32)
+    di, dc = torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
+    L = BlockLists()
+    L.idx, L.cnt, L.cap, L.head_shared = di.data_ptr(), dc.data_ptr(), 4, 0
+    prm = AttnParams()
+    prm.mode, prm.block_q, prm.kv_unit, prm.scale = 0, 128, 32, 0.0
+    o = torch.empty(q.shape, dtype=q.dtype, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    api.sta_sparse_attn_fwd(session.problem(w), prm, q.cuda(), k.cuda(), v.cuda(), L, o,
+                            dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & _lib.STA_DEV_BAD_INDEX
+    oc = o.cpu()
+    for qb in range(4):
+        units = [u for u in idx[qb, :cnt[qb]].tolist() if 0 <= u < n_units]
+        lo, hi = qb * 128, min(w["N"], qb * 128 + 128)
+        ref = block_sparse_rows(q[0], k[0], v[0], qb, units, 128, 32)
+        assert_close_attn(oc[0, lo:hi].float().numpy(), ref, f"qb {qb}")

@@ -69,3 +69,10 @@ def test_host_argument_checks(lib):
                                    None) == STA_ERR_UNSUPPORTED
     assert lib.sta_build_blocks_rows(ctypes.byref(good), ctypes.byref(sel)) == 2
     assert lib.sta_attn_workspace(ctypes.byref(Problem(2, 4, 8, 8, 64, 1))) == 3 * 2 * 256 * 64 * 2
+
+
+def test_selftest_argument_checks(lib):
+    from sparse_spatiotemporal_attention_video_b200._lib import STA_ERR_ARG
+    assert lib.sta_selftest_bounded_wait(0, 1, 1, None) == STA_ERR_ARG
+    assert lib.sta_selftest_bounded_wait(10**10, 1, 1, None) == STA_ERR_ARG
+    assert lib.sta_selftest_bounded_wait(1000, None, 1, None) == STA_ERR_ARG
