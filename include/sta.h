@@ -66,6 +66,7 @@ typedef enum {
 #define STA_DEV_CAPACITY  0x2  /* a list row was truncated at `cap`                  */
 #define STA_DEV_EMPTY_ROW 0x4  /* a query row had no kept key; its output is 0      */
 #define STA_DEV_BAD_INDEX 0x8  /* a list entry was out of range and was skipped     */
+#define STA_DEV_RANGE     0x10 /* an importance operand exceeded the fp16 range     */
 
 typedef enum { STA_BF16 = 0, STA_F32 = 1 } sta_dtype;
 
@@ -157,7 +158,9 @@ typedef struct {
   int32_t* radius;
 } sta_block_lists;
 
-/* Workspace bytes sta_build_blocks needs for this problem and selector. */
+/* Workspace bytes sta_build_blocks needs for this problem and selector.
+ * The workspace must start on a 256-byte boundary (cudaMalloc and torch
+ * allocations do); any other start is STA_ERR_WORKSPACE. */
 size_t sta_build_blocks_workspace(const sta_problem* prob, const sta_selector_params* sel);
 
 /* Rows of the lists the selector writes (n_qblocks, or heads*n_qblocks). */

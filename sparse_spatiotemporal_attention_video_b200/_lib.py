@@ -19,6 +19,7 @@ STA_DEV_TIMEOUT = 0x1
 STA_DEV_CAPACITY = 0x2
 STA_DEV_EMPTY_ROW = 0x4
 STA_DEV_BAD_INDEX = 0x8
+STA_DEV_RANGE = 0x10
 
 STA_BF16, STA_F32 = 0, 1
 STA_SEL_RADIAL, STA_SEL_ENTROPY, STA_SEL_IBCS_SIP, STA_SEL_ROUTED = 0, 1, 2, 3

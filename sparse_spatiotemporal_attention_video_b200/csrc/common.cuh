@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <atomic>
@@ -113,13 +114,21 @@ cudaError_t launch_routed_local_lists(int F, int H, int W, int B, int U, int win
                                       int32_t* required_cap, int32_t* dev_status,
                                       cudaStream_t s);
 
-// Clustering importance + inclusion-probability sampling (sel_ibcs.cu).
+// Clustering importance + inclusion-probability sampling (sel_ibcs.cu,
+// sel_importance.cu).
 int ibcs_max_subblocks();
-cudaError_t launch_ibcs_sip(const __nv_bfloat16* q, const float* kbar, float* cent, float* wts,
-                            float* z, float* stats, int heads, int N, int d, int B, int U, int km_k, int iters,
-                            int m, uint64_t seed, float scale, int32_t* idx, float* logw,
-                            int32_t* cnt, int cap, int32_t* required_cap, int32_t* dev_status,
-                            cudaStream_t s);
+cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
+                          int d, int B, int km_k, int iters, cudaStream_t s);
+cudaError_t launch_split_f16(const float* x, __half* hi, __half* lo, size_t n,
+                             int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_importance_tc(const float* wts, float* p, int heads, int n_rows, int nqb,
+                                 int km, int n_sub, int N, int U, float scale,
+                                 const CUtensorMap& ch,
+                                 const CUtensorMap& cl, const CUtensorMap& kh,
+                                 const CUtensorMap& kl, int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_sip_sample(const float* p, int rows, int n_sub, int m, uint64_t seed,
+                              int32_t* idx, float* logw, int32_t* cnt, int cap,
+                              int32_t* required_cap, int32_t* dev_status, cudaStream_t s);
 
 // Self-test of the bounded wait (selftest.cu).
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* dev_status,

@@ -21,7 +21,7 @@
 //     empty cluster keeps its centroid); n_c = member counts of the last
 //     assignment.                                           (kmeans_kernel)
 //  3. p_j = sum_c (n_c / n_b) softmax_j(c_c . Kbar_j * scale + ln n_j)
-//                                                       (importance_kernel)
+//                          (importance_tc_kernel in sel_importance.cu)
 //  4. m = ceil(frac * n_sub) (host); pi_j = min(1, lambda p_j) with
 //     sum_j pi_j = m by water filling: repeatedly set lambda = (m - #capped)
 //     / (sum of uncapped p) and cap every j with lambda p_j >= 1.
@@ -30,9 +30,9 @@
 //     logw_j = -ln pi_j.                                  (sip_sample_kernel)
 //
 // Precision: the sampling decisions compare u_j with pi_j, so p is computed
-// to fp32 accuracy (fp32 scores on the FMA pipe, fp64 sums of the softmax
-// normaliser and of the water-filling sums) rather than on the bf16 tensor
-// cores, whose logit error would move pi by ~1e-3.
+// to fp32 accuracy: the importance scores on the tensor cores from fp16
+// hi/lo operand splits (sel_importance.cu), fp64 sums of the softmax
+// normaliser and of the water-filling sums.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -179,197 +179,6 @@ __global__ void __launch_bounds__(kKmThreads) kmeans_kernel(
   }
 }
 
-// --------------------------------------------------------------- importance
-// CTA tile: 128 centroid rows (128/KM query blocks of one head) x 128
-// sub-blocks, K = D in chunks of 32.  The centroid tile is staged once,
-// transposed (As[k][row]); sub-block-mean chunks are double-buffered through
-// registers (Bs[k][j]).  Thread (ty, tx) owns rows ty*8..ty*8+7 (8/KM whole
-// query blocks) and columns tx*4..tx*4+3 and 64+tx*4..64+tx*4+3 (two float4
-// reads per k that fall on distinct banks).  One sweep over all sub-blocks
-// stores the scores z_cj and keeps an online max and an fp64 sum of exp per
-// row; the 16 threads of a row group then merge them into (w_c / Z_c, M_c).
-// Storing z (4 B per score, written and read once) is cheaper than a second
-// sweep of the GEMM; sip_sample_kernel forms p from it.
-constexpr int kImpThreads = 256;
-constexpr int kImpRows = 128;
-constexpr int kImpCols = 128;
-constexpr int kImpKc = 32;
-constexpr int kImpPad = 4;
-constexpr int kImpStride = kImpCols + kImpPad;
-
-template <int D>
-constexpr size_t imp_smem_bytes() {
-  return sizeof(float) * (static_cast<size_t>(D) * (kImpRows + kImpPad) +
-                          2ull * kImpKc * kImpStride);
-}
-
-template <int D, int KM>
-__global__ void __launch_bounds__(kImpThreads, 1) importance_kernel(
-    const float* __restrict__ cent, const float* __restrict__ wts,
-    const float* __restrict__ kbar, int nqb, int n_sub, int N, int U, float scale,
-    float* __restrict__ zout, float* __restrict__ stats) {
-  static_assert(8 % KM == 0, "centroids per query block must divide 8");
-  constexpr int NCH = D / kImpKc;
-  extern __shared__ float4 imp_smem4[];
-  float* As = reinterpret_cast<float*>(imp_smem4);     // [D][kImpRows + pad]
-  float* Bs = As + D * (kImpRows + kImpPad);           // [2][kImpKc][kImpStride]
-  const int head = blockIdx.y;
-  const int row0 = blockIdx.x * kImpRows;              // first centroid row (per head)
-  const int n_rows = nqb * KM;
-  const int tid = threadIdx.x;
-  const int ty = tid >> 4, tx = tid & 15;
-  const float* ch = cent + static_cast<size_t>(head) * n_rows * D;
-  const float* kh = kbar + static_cast<size_t>(head) * n_sub * D;
-
-  for (int i = tid; i < kImpRows * (D / 4); i += kImpThreads) {
-    const int r = i % kImpRows, k4 = i / kImpRows;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (row0 + r < n_rows) v = reinterpret_cast<const float4*>(ch + static_cast<size_t>(row0 + r) * D)[k4];
-    As[(4 * k4 + 0) * (kImpRows + kImpPad) + r] = v.x;
-    As[(4 * k4 + 1) * (kImpRows + kImpPad) + r] = v.y;
-    As[(4 * k4 + 2) * (kImpRows + kImpPad) + r] = v.z;
-    As[(4 * k4 + 3) * (kImpRows + kImpPad) + r] = v.w;
-  }
-
-  // B chunk loader: 32 k x 128 j = 1024 float4, 4 per thread
-  auto load_chunk = [&](int j0, int ch_i, float4 (&reg)[4]) {
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int i = tid + t * kImpThreads;
-      const int j = i % kImpCols, k4 = i / kImpCols;
-      reg[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j0 + j < n_sub)
-        reg[t] = reinterpret_cast<const float4*>(kh + static_cast<size_t>(j0 + j) * D +
-                                                 ch_i * kImpKc)[k4];
-    }
-  };
-  auto store_chunk = [&](int buf, const float4 (&reg)[4]) {
-    float* b = Bs + buf * kImpKc * kImpStride;
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const int i = tid + t * kImpThreads;
-      const int j = i % kImpCols, k4 = i / kImpCols;
-      b[(4 * k4 + 0) * kImpStride + j] = reg[t].x;
-      b[(4 * k4 + 1) * kImpStride + j] = reg[t].y;
-      b[(4 * k4 + 2) * kImpStride + j] = reg[t].z;
-      b[(4 * k4 + 3) * kImpStride + j] = reg[t].w;
-    }
-  };
-  // z[8][8] = scores of this thread's rows x columns for sub-block tile j0
-  auto tile_scores = [&](int j0, float (&z)[8][8]) {
-#pragma unroll
-    for (int a = 0; a < 8; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) z[a][b] = 0.f;
-    float4 reg[4];
-    load_chunk(j0, 0, reg);
-    __syncthreads();  // previous users of Bs are done
-    store_chunk(0, reg);
-    __syncthreads();
-#pragma unroll 1
-    for (int c = 0; c < NCH; ++c) {
-      if (c + 1 < NCH) load_chunk(j0, c + 1, reg);
-      const float* b = Bs + (c & 1) * kImpKc * kImpStride;
-#pragma unroll 4
-      for (int kk = 0; kk < kImpKc; ++kk) {
-        const float* ar = As + (c * kImpKc + kk) * (kImpRows + kImpPad) + ty * 8;
-        const float4 a0 = *reinterpret_cast<const float4*>(ar);
-        const float4 a1 = *reinterpret_cast<const float4*>(ar + 4);
-        const float4 b0 = *reinterpret_cast<const float4*>(b + kk * kImpStride + tx * 4);
-        const float4 b1 = *reinterpret_cast<const float4*>(b + kk * kImpStride + 64 + tx * 4);
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-        for (int x = 0; x < 8; ++x)
-#pragma unroll
-          for (int y = 0; y < 8; ++y) z[x][y] = fmaf(av[x], bv[y], z[x][y]);
-      }
-      if (c + 1 < NCH) {
-        store_chunk((c + 1) & 1, reg);
-        __syncthreads();
-      }
-    }
-    // scale and ln n_j; columns past n_sub are -inf
-#pragma unroll
-    for (int y = 0; y < 8; ++y) {
-      const int j = j0 + (y < 4 ? tx * 4 + y : 64 + tx * 4 + (y - 4));
-      float lnn = -INFINITY;
-      if (j < n_sub) lnn = logf(static_cast<float>(min(U, N - j * U)));
-#pragma unroll
-      for (int x = 0; x < 8; ++x) z[x][y] = (j < n_sub) ? fmaf(z[x][y], scale, lnn) : -INFINITY;
-    }
-  };
-
-  // ---- sweep 1: per-row max and sum of exp
-  float m[8];
-  double s[8];
-#pragma unroll
-  for (int x = 0; x < 8; ++x) {
-    m[x] = -INFINITY;
-    s[x] = 0.0;
-  }
-  for (int j0 = 0; j0 < n_sub; j0 += kImpCols) {
-    float z[8][8];
-    tile_scores(j0, z);
-    // keep the scores: p is formed from them once the normalisers are known
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const int r = row0 + ty * 8 + x;
-      if (r >= n_rows) continue;
-      float* zr = zout + (static_cast<size_t>(head) * n_rows + r) * n_sub + j0;
-#pragma unroll
-      for (int y = 0; y < 8; ++y) {
-        const int c = y < 4 ? tx * 4 + y : 64 + tx * 4 + (y - 4);
-        if (j0 + c < n_sub) zr[c] = z[x][y];
-      }
-    }
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      float t = z[x][0];
-#pragma unroll
-      for (int y = 1; y < 8; ++y) t = fmaxf(t, z[x][y]);
-      if (t == -INFINITY) continue;
-      if (t > m[x]) {
-        if (m[x] != -INFINITY) s[x] *= exp(static_cast<double>(m[x]) - static_cast<double>(t));
-        m[x] = t;
-      }
-      double acc = 0.0;
-#pragma unroll
-      for (int y = 0; y < 8; ++y) acc += static_cast<double>(expf(z[x][y] - m[x]));
-      s[x] += acc;
-    }
-  }
-  // merge the 16 column groups of each row group (lanes with equal ty)
-#pragma unroll
-  for (int x = 0; x < 8; ++x) {
-#pragma unroll
-    for (int o = 1; o < 16; o <<= 1) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[x], o);
-      const double so = __shfl_xor_sync(0xffffffffu, s[x], o);
-      const float mn = fmaxf(m[x], mo);
-      double acc = 0.0;
-      if (m[x] != -INFINITY) acc += s[x] * exp(static_cast<double>(m[x]) - static_cast<double>(mn));
-      if (mo != -INFINITY) acc += so * exp(static_cast<double>(mo) - static_cast<double>(mn));
-      m[x] = mn;
-      s[x] = acc;
-    }
-  }
-  // per centroid row: coefficient w_c / Z_c and the maximum M_c
-  if (tx == 0) {
-#pragma unroll
-    for (int x = 0; x < 8; ++x) {
-      const int r = row0 + ty * 8 + x;
-      if (r >= n_rows) continue;
-      float coef = 0.f;
-      if (s[x] > 0.0)
-        coef = static_cast<float>(
-            static_cast<double>(__ldg(wts + static_cast<size_t>(head) * n_rows + r)) / s[x]);
-      float2* st = reinterpret_cast<float2*>(stats) + static_cast<size_t>(head) * n_rows + r;
-      *st = make_float2(coef, m[x]);
-    }
-  }
-}
-
 // ------------------------------------------------------------ SIP sampling
 constexpr int kSipThreads = 256;
 constexpr int kSipWarps = kSipThreads / 32;
@@ -426,46 +235,20 @@ __device__ __forceinline__ int block_sum_i(int v, int* red, int& excl) {
   return tot;
 }
 
-template <int KM>
 __global__ void __launch_bounds__(kSipThreads) sip_sample_kernel(
-    const float* __restrict__ z, const float* __restrict__ stats, int n_sub, int m,
-    uint32_t seed_lo, uint32_t seed_hi, int32_t* __restrict__ idx, float* __restrict__ logw,
-    int32_t* __restrict__ cnt, int cap, int32_t* required_cap, int32_t* dev_status) {
+    const float* __restrict__ p, int n_sub, int m, uint32_t seed_lo, uint32_t seed_hi,
+    int32_t* __restrict__ idx, float* __restrict__ logw, int32_t* __restrict__ cnt, int cap,
+    int32_t* required_cap, int32_t* dev_status) {
   extern __shared__ float sip_smem[];
   float* sp = sip_smem;                                    // [n_sub]
   uint8_t* capped = reinterpret_cast<uint8_t*>(sp + n_sub);  // [n_sub]
   __shared__ double redd[kSipWarps];
   __shared__ int redi[kSipWarps];
-  __shared__ float2 cs[KM];
   const int row = blockIdx.x;  // head * nqb + qb
-  if (threadIdx.x < KM)
-    cs[threadIdx.x] = reinterpret_cast<const float2*>(stats)[static_cast<size_t>(row) * KM + threadIdx.x];
-  __syncthreads();
-  // p_j = sum_c (w_c / Z_c) exp(z_cj - M_c), centroids in order; the scores
-  // of four j per thread are loaded before any is used
-  const float* zr = z + static_cast<size_t>(row) * KM * n_sub;
-  for (int j0 = threadIdx.x; j0 < n_sub; j0 += 4 * kSipThreads) {
-    float zv[4][KM];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = j0 + u * kSipThreads;
-#pragma unroll
-      for (int c = 0; c < KM; ++c)
-        zv[u][c] = j < n_sub ? __ldcs(zr + static_cast<size_t>(c) * n_sub + j) : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = j0 + u * kSipThreads;
-      if (j >= n_sub) break;
-      float acc = 0.f;
-#pragma unroll
-      for (int c = 0; c < KM; ++c) {
-        const float2 cm = cs[c];
-        if (cm.x != 0.f) acc = fmaf(cm.x, expf(zv[u][c] - cm.y), acc);
-      }
-      sp[j] = acc;
-      capped[j] = 0;
-    }
+  const float* pr = p + static_cast<size_t>(row) * ((n_sub + 3) & ~3);  // 16-byte rows
+  for (int j = threadIdx.x; j < n_sub; j += kSipThreads) {
+    sp[j] = __ldcs(pr + j);
+    capped[j] = 0;
   }
   __syncthreads();
   // water filling
@@ -541,34 +324,15 @@ __global__ void __launch_bounds__(kSipThreads) sip_sample_kernel(
 }
 
 template <int D, int KM>
-cudaError_t launch_ibcs_t(const __nv_bfloat16* q, const float* kbar, float* cent, float* wts,
-                          float* z, float* stats, int heads, int N, int B, int U, int iters, int m,
-                          uint64_t seed, float scale, int32_t* idx, float* logw, int32_t* cnt,
-                          int cap, int32_t* required_cap, int32_t* dev_status, cudaStream_t s) {
+cudaError_t launch_kmeans_t(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
+                            int B, int iters, cudaStream_t s) {
   const int nqb = (N + B - 1) / B;
-  const int n_sub = (N + U - 1) / U;
   const size_t km_smem =
       sizeof(float) * (static_cast<size_t>(kKmRows) * (D + 1) + KM * D + 4 * kKmRows * KM) +
       sizeof(int) * (kKmRows + 4 * KM);
   cudaError_t e = set_dyn_smem<kmeans_kernel<D, KM>>(static_cast<int>(km_smem));
   if (e != cudaSuccess) return e;
   kmeans_kernel<D, KM><<<heads * nqb, kKmThreads, km_smem, s>>>(q, N, B, nqb, iters, cent, wts);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-  const size_t imp_smem = imp_smem_bytes<D>();
-  e = set_dyn_smem<importance_kernel<D, KM>>(static_cast<int>(imp_smem));
-  if (e != cudaSuccess) return e;
-  dim3 gi((nqb * KM + kImpRows - 1) / kImpRows, heads);
-  importance_kernel<D, KM><<<gi, kImpThreads, imp_smem, s>>>(cent, wts, kbar, nqb, n_sub, N, U,
-                                                             scale, z, stats);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-  const size_t sip_smem = static_cast<size_t>(n_sub) * (sizeof(float) + 1);
-  e = set_dyn_smem<sip_sample_kernel<KM>>(static_cast<int>(sip_smem));
-  if (e != cudaSuccess) return e;
-  sip_sample_kernel<KM><<<heads * nqb, kSipThreads, sip_smem, s>>>(
-      z, stats, n_sub, m, static_cast<uint32_t>(seed & 0xffffffffu), static_cast<uint32_t>(seed >> 32),
-      idx, logw, cnt, cap, required_cap, dev_status);
   return cudaGetLastError();
 }
 
@@ -576,25 +340,32 @@ cudaError_t launch_ibcs_t(const __nv_bfloat16* q, const float* kbar, float* cent
 
 int ibcs_max_subblocks() { return static_cast<int>((200 * 1024) / (sizeof(float) + 1)); }
 
-cudaError_t launch_ibcs_sip(const __nv_bfloat16* q, const float* kbar, float* cent, float* wts,
-                            float* z, float* stats, int heads, int N, int d, int B, int U, int km_k, int iters,
-                            int m, uint64_t seed, float scale, int32_t* idx, float* logw,
-                            int32_t* cnt, int cap, int32_t* required_cap, int32_t* dev_status,
-                            cudaStream_t s) {
-#define STA_IBCS_CASE(DD, KK)                                                                   \
-  if (d == DD && km_k == KK)                                                                    \
-    return launch_ibcs_t<DD, KK>(q, kbar, cent, wts, z, stats, heads, N, B, U, iters, m, seed, scale, \
-                                 idx, logw, cnt, cap, required_cap, dev_status, s);
-  STA_IBCS_CASE(128, 4)
-  STA_IBCS_CASE(128, 2)
-  STA_IBCS_CASE(128, 1)
-  STA_IBCS_CASE(128, 8)
-  STA_IBCS_CASE(64, 4)
-  STA_IBCS_CASE(64, 2)
-  STA_IBCS_CASE(64, 1)
-  STA_IBCS_CASE(64, 8)
-#undef STA_IBCS_CASE
+cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
+                          int d, int B, int km_k, int iters, cudaStream_t s) {
+#define STA_KM_CASE(DD, KK) \
+  if (d == DD && km_k == KK) return launch_kmeans_t<DD, KK>(q, cent, wts, heads, N, B, iters, s);
+  STA_KM_CASE(128, 4)
+  STA_KM_CASE(128, 2)
+  STA_KM_CASE(128, 1)
+  STA_KM_CASE(128, 8)
+  STA_KM_CASE(64, 4)
+  STA_KM_CASE(64, 2)
+  STA_KM_CASE(64, 1)
+  STA_KM_CASE(64, 8)
+#undef STA_KM_CASE
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_sip_sample(const float* p, int rows, int n_sub, int m, uint64_t seed,
+                              int32_t* idx, float* logw, int32_t* cnt, int cap,
+                              int32_t* required_cap, int32_t* dev_status, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(n_sub) * (sizeof(float) + 1);
+  cudaError_t e = set_dyn_smem<sip_sample_kernel>(static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  sip_sample_kernel<<<rows, kSipThreads, smem, s>>>(
+      p, n_sub, m, static_cast<uint32_t>(seed & 0xffffffffu), static_cast<uint32_t>(seed >> 32),
+      idx, logw, cnt, cap, required_cap, dev_status);
+  return cudaGetLastError();
 }
 
 }  // namespace sta

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <math.h>
+#include <stdint.h>
 
 #include <mutex>
 
@@ -42,7 +43,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // 3D map over a [heads][N][d] bf16 tensor: dim0 = d (contiguous), dim1 = N,
 // dim2 = heads; box = 64 columns (128 bytes, 128-byte swizzle) x rows x 1.
 // Rows past N read as zero.
-bool make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_rows) {
+bool make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box_rows,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
@@ -51,7 +53,7 @@ bool make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box
                            static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+  CUresult r = enc(m, dtype, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -137,7 +139,8 @@ sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16*
 
 // Workspace carve-up of the content selectors (256-byte aligned segments).
 struct SelWorkspace {
-  size_t qbar = 0, kbar = 0, scores = 0, cent = 0, wts = 0, z = 0, stats = 0, total = 0;
+  size_t qbar = 0, kbar = 0, scores = 0, cent = 0, wts = 0, p = 0;
+  size_t kb_hi = 0, kb_lo = 0, c_hi = 0, c_lo = 0, total = 0;
 };
 
 SelWorkspace sel_workspace(const sta_problem* p, const sta_selector_params* sel) {
@@ -161,10 +164,13 @@ SelWorkspace sel_workspace(const sta_problem* p, const sta_selector_params* sel)
   } else if (sel->kind == STA_SEL_IBCS_SIP) {
     const size_t km = sel->km_k > 0 ? static_cast<size_t>(sel->km_k) : 1;
     w.kbar = take(h * nku * d * 4);
+    w.kb_hi = take(h * nku * d * 2);
+    w.kb_lo = take(h * nku * d * 2);
     w.cent = take(h * nqb * km * d * 4);
+    w.c_hi = take(h * nqb * km * d * 2);
+    w.c_lo = take(h * nqb * km * d * 2);
     w.wts = take(h * nqb * km * 4);
-    w.z = take(h * nqb * km * nku * 4);
-    w.stats = take(h * nqb * km * 8);
+    w.p = take(h * nqb * ((nku + 3) & ~size_t(3)) * 4);  // rows padded to 16 bytes
   }
   w.total = off;
   return w;
@@ -215,6 +221,7 @@ const char* sta_dev_status_string(int32_t bits) {
   if (bits == 0) return "ok";
   if (bits & STA_DEV_TIMEOUT) return "timeout: a bounded wait ran out";
   if (bits & STA_DEV_BAD_INDEX) return "list entry out of range (skipped)";
+  if (bits & STA_DEV_RANGE) return "importance operand beyond the fp16 range";
   if (bits & STA_DEV_CAPACITY) return "list row truncated at capacity";
   if (bits & STA_DEV_EMPTY_ROW) return "query row without kept keys (output 0)";
   return "unknown device status";
@@ -274,7 +281,9 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
           (prob->W - 1) / sel->ent_tile_w > 1023)
         return STA_ERR_UNSUPPORTED;
       const SelWorkspace w = sel_workspace(prob, sel);
-      if (!workspace || workspace_bytes < w.total) return STA_ERR_WORKSPACE;
+      if (!workspace || workspace_bytes < w.total ||
+          (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return STA_ERR_WORKSPACE;
       uint8_t* ws = static_cast<uint8_t*>(workspace);
       float* qbar = reinterpret_cast<float*>(ws + w.qbar);
       float* kbar = reinterpret_cast<float*>(ws + w.kbar);
@@ -316,28 +325,54 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       if (sel->km_k != 1 && sel->km_k != 2 && sel->km_k != 4 && sel->km_k != 8)
         return STA_ERR_UNSUPPORTED;
       if (sel->km_iters < 1) return STA_ERR_ARG;
+      if (prob->d != 128) return STA_ERR_UNSUPPORTED;  // tensor-core importance: d = 128
       if (!(sel->sample_frac > 0.f && sel->sample_frac <= 1.f)) return STA_ERR_ARG;
       const int N = prob->F * prob->H * prob->W;
       const int n_sub = (N + sel->kv_unit - 1) / sel->kv_unit;
       if (n_sub > ibcs_max_subblocks()) return STA_ERR_UNSUPPORTED;
       const SelWorkspace w = sel_workspace(prob, sel);
-      if (!workspace || workspace_bytes < w.total) return STA_ERR_WORKSPACE;
+      if (!workspace || workspace_bytes < w.total ||
+          (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return STA_ERR_WORKSPACE;
       uint8_t* ws = static_cast<uint8_t*>(workspace);
       float* kbar = reinterpret_cast<float*>(ws + w.kbar);
       float* cent = reinterpret_cast<float*>(ws + w.cent);
       float* wts = reinterpret_cast<float*>(ws + w.wts);
-      float* zbuf = reinterpret_cast<float*>(ws + w.z);
-      float* sbuf = reinterpret_cast<float*>(ws + w.stats);
+      float* pbuf = reinterpret_cast<float*>(ws + w.p);
+      __half* kbh = reinterpret_cast<__half*>(ws + w.kb_hi);
+      __half* kbl = reinterpret_cast<__half*>(ws + w.kb_lo);
+      __half* ch = reinterpret_cast<__half*>(ws + w.c_hi);
+      __half* cl = reinterpret_cast<__half*>(ws + w.c_lo);
       out->head_shared = 0;
       const int m = fraction_count(sel->sample_frac, n_sub, 1);
       const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
+      const int nqb = (N + sel->block_q - 1) / sel->block_q;
+      const int n_rows = nqb * sel->km_k;
+      const size_t nk = static_cast<size_t>(prob->heads) * n_sub * prob->d;
+      const size_t nc = static_cast<size_t>(prob->heads) * n_rows * prob->d;
+      // 1. sub-block means, 2. k-means, 3. fp16 hi/lo splits
       if (failed(launch_block_means(static_cast<const __nv_bfloat16*>(k), nullptr, kbar, nullptr,
-                             prob->heads, N, prob->d, sel->kv_unit, s)))
+                                    prob->heads, N, prob->d, sel->kv_unit, s)) ||
+          failed(launch_kmeans(static_cast<const __nv_bfloat16*>(q), cent, wts, prob->heads, N,
+                               prob->d, sel->block_q, sel->km_k, sel->km_iters, s)) ||
+          failed(launch_split_f16(kbar, kbh, kbl, nk, dev_status, s)) ||
+          failed(launch_split_f16(cent, ch, cl, nc, dev_status, s)))
         return STA_ERR_CUDA;
-      if (failed(launch_ibcs_sip(static_cast<const __nv_bfloat16*>(q), kbar, cent, wts, zbuf, sbuf,
-                          prob->heads, N, prob->d, sel->block_q, sel->kv_unit, sel->km_k,
-                          sel->km_iters, m, sel->seed, scale, out->idx, out->logw, out->cnt,
-                          out->cap, out->required_cap, dev_status, s)))
+      // 4. importance on the tensor cores, 5. water filling + Philox sampling
+      CUtensorMap tch, tcl, tkh, tkl;
+      if (!make_map(&tch, ch, prob->d, n_rows, prob->heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+          !make_map(&tcl, cl, prob->d, n_rows, prob->heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+          !make_map(&tkh, kbh, prob->d, n_sub, prob->heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+          !make_map(&tkl, kbl, prob->d, n_sub, prob->heads, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16)) {
+        g_last_cuda_error = cudaErrorInvalidValue;
+        return STA_ERR_CUDA;
+      }
+      if (failed(launch_importance_tc(wts, pbuf, prob->heads, n_rows, nqb, sel->km_k, n_sub, N,
+                                      sel->kv_unit,
+                                      scale, tch, tcl, tkh, tkl, dev_status, s)) ||
+          failed(launch_sip_sample(pbuf, prob->heads * nqb, n_sub, m, sel->seed, out->idx,
+                                   out->logw, out->cnt, out->cap, out->required_cap, dev_status,
+                                   s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }

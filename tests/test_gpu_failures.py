@@ -88,3 +88,26 @@ def test_out_of_range_entry_is_skipped_and_flagged(cuda_ok):
         lo, hi = qb * 128, min(w["N"], qb * 128 + 128)
         ref = block_sparse_rows(q[0], k[0], v[0], qb, units, 128, 32)
         assert_close_attn(oc[0, lo:hi].float().numpy(), ref, f"qb {qb}")
+
+
+def test_misaligned_workspace_is_rejected(cuda_ok):
+    """The selector workspace must start on a 256-byte boundary (its segments
+    feed TMA descriptors and 16-byte stores); another start is an argument
+    error reported before any launch."""
+    _lib, api, session = _mods()
+    w = workload("ab_sampled", heads=1, F=2, H=8, W=16)
+    q, k, _ = make_qkv(w)
+    need = api.sta_build_blocks_workspace(session.problem(w), session.selector(w))
+    ws = torch.empty(need + 512, dtype=torch.uint8, device="cuda")
+    L = session.Lists(w)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with pytest.raises(_lib.StaError) as e:
+        api.sta_build_blocks(session.problem(w), session.selector(w), q.cuda(), k.cuda(),
+                             L.struct, workspace=ws.data_ptr() + 16, workspace_bytes=need,
+                             dev_status=st)
+    assert e.value.code == _lib.STA_ERR_WORKSPACE
+    # the aligned start of the same buffer works
+    api.sta_build_blocks(session.problem(w), session.selector(w), q.cuda(), k.cuda(), L.struct,
+                         workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
