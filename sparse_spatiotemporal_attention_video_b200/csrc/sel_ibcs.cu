@@ -43,139 +43,192 @@ namespace sta {
 namespace {
 
 // ------------------------------------------------------------------ k-means
-// One CTA of 512 threads per (head, query block).  Assignment: thread
-// (g, r) = (tid / 128, tid % 128) sums the squared distance of query r over
-// dimension quarter g; the four partials are added in order g = 0..3.
-// Update: thread (g, r) sums dimension r over queries [32g, 32g+32) per
-// cluster; the four partials are added in order.  Rows of the staged block
-// have an odd stride (D+1 floats), so the 32 lanes of a warp (consecutive r)
-// hit distinct banks.
-constexpr int kKmThreads = 512;
-constexpr int kKmRows = 128;  // largest query block
+// One CTA of 256 threads per (head, query block), the block staged once in
+// shared memory as bf16 (exact) and its fp32 values held in registers.
+//
+// Assignment: thread (g, p) = (tid / 64, tid % 64) owns queries p and p + 64
+// over dimension quarter g (32 fp32 values each, in registers for all
+// iterations) and forms the partial squared distances to every centroid
+// with packed f32x2 subtract / fused multiply-add (even and odd dimensions
+// in the two halves, added at the end); the centroids are read from shared
+// memory as warp-uniform 16-byte broadcasts.  The four quarter partials of a
+// query are added in order g = 0..3 and the argmin keeps the lower index on
+// ties.  The direct form sum (x - c)^2 is kept (not |c|^2 - 2 x.c): it has no
+// cancellation, so the distance carries fp32 rounding relative to itself.
+//
+// Update: the members are counting-sorted by cluster (warp ballots), so the
+// member sum of dimension pair j over cluster c is a run of plain adds; thread
+// (s, j) = (tid / 64, tid % 64) sums dimension pair j over the quarter s of
+// the sorted members, cut at cluster boundaries, and the four partials are
+// added in order.  An empty cluster keeps its centroid.
+constexpr int kKmThreads = 256;
+constexpr int kKmRows = 128;           // largest query block
+constexpr int kKmRowPitch = 128 + 8;   // bf16 per staged row (272 B: conflict-free 16 B reads)
 
-template <int D, int KM>
-__global__ void __launch_bounds__(kKmThreads) kmeans_kernel(
+template <int KM>
+struct KmSmem {
+  __nv_bfloat16 q[kKmRows * kKmRowPitch];  // staged block, rows >= nb zero
+  float negc[KM * 128];                    // -centroid
+  float part[4 * KM * kKmRows];            // [g][c][r] distances / [s][c][dim] sums
+  int perm[kKmRows];                       // members sorted by cluster
+  int wcount[4][KM];                       // per-warp member counts (warps 0-3)
+  int start[KM + 1];                       // first sorted position of each cluster
+};
+
+template <int KM>
+__global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 1 : 2) kmeans_kernel(
     const __nv_bfloat16* __restrict__ q, int N, int B, int nqb, int iters,
     float* __restrict__ cent, float* __restrict__ wts) {
-  constexpr int QS = D + 1;
-  constexpr int DQ = D / 4;  // dimensions per quarter
-  extern __shared__ float km_smem[];
-  float* sq = km_smem;                       // [128][QS]
-  float* sc = sq + kKmRows * QS;             // [KM][D]
-  float* part = sc + KM * D;                 // [4][128][KM] distances / [4][KM][D] sums
-  int* sassign = reinterpret_cast<int*>(part + 4 * kKmRows * KM);  // [128]
-  int* pcount = sassign + kKmRows;           // [4][KM]
-  __shared__ int scount[KM];
+  constexpr int D = 128;
+  extern __shared__ __align__(16) uint8_t km_raw[];
+  KmSmem<KM>& sm = *reinterpret_cast<KmSmem<KM>*>(km_raw);
+  const int tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;  // head * nqb + qb
   const int head = row / nqb;
   const int qb = row - head * nqb;
   const int q0 = qb * B;
   const int nb = min(B, N - q0);
-  const int g = threadIdx.x / kKmRows;
-  const int r = threadIdx.x - g * kKmRows;
   const __nv_bfloat16* qh = q + (static_cast<size_t>(head) * N + q0) * D;
-  // stage the block as fp32 (rows >= nb are never read)
-  for (int i = threadIdx.x; i < nb * D / 8; i += kKmThreads) {
-    const int rr = (i * 8) / D;
-    const int c = i * 8 - rr * D;
-    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(qh) + i);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      sq[rr * QS + c + 2 * t] = __uint_as_float(w[t] << 16);
-      sq[rr * QS + c + 2 * t + 1] = __uint_as_float(w[t] & 0xffff0000u);
-    }
+
+  // stage the block (16-byte loads, 16 per row); rows >= nb are zero
+  for (int i = tid; i < kKmRows * (D / 8); i += kKmThreads) {
+    const int r = i >> 4, c8 = (i & 15) * 8;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < nb) v = __ldcs(reinterpret_cast<const uint4*>(qh) + i);
+    *reinterpret_cast<uint4*>(&sm.q[r * kKmRowPitch + c8]) = v;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < KM * D; i += kKmThreads) {
+  for (int i = tid; i < KM * D; i += kKmThreads) {
     const int c = i / D, col = i - c * D;
-    sc[i] = sq[((c * nb) / KM) * QS + col];
+    sm.negc[i] = -__bfloat162float(sm.q[((c * nb) / KM) * kKmRowPitch + col]);
+  }
+  // registers: queries p and p + 64, dimensions [32g, 32g + 32) as 16 pairs
+  const int g = tid >> 6, p = tid & 63;
+  float2 x[2][16];
+#pragma unroll
+  for (int qi = 0; qi < 2; ++qi) {
+#pragma unroll
+    for (int v8 = 0; v8 < 4; ++v8) {
+      const uint4 w =
+          *reinterpret_cast<const uint4*>(&sm.q[(p + 64 * qi) * kKmRowPitch + 32 * g + 8 * v8]);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        x[qi][4 * v8 + t] = make_float2(__uint_as_float(ww[t] << 16),
+                                        __uint_as_float(ww[t] & 0xffff0000u));
+    }
   }
   __syncthreads();
+
   for (int it = 0; it < iters; ++it) {
-    // assignment: partial squared distances over one quarter of the dims
-    if (r < nb) {
-      float d2[KM];
+    // ---- assignment: partial distances over quarter g
+    {
+      float2 acc[2][KM];
 #pragma unroll
-      for (int c = 0; c < KM; ++c) d2[c] = 0.f;
-#pragma unroll 8
-      for (int i = 0; i < DQ; ++i) {
-        const int col = g * DQ + i;
-        const float x = sq[r * QS + col];
+      for (int qi = 0; qi < 2; ++qi)
 #pragma unroll
-        for (int c = 0; c < KM; ++c) {
-          const float t = x - sc[c * D + col];
-          d2[c] = fmaf(t, t, d2[c]);
-        }
-      }
+        for (int c = 0; c < KM; ++c) acc[qi][c] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int c = 0; c < KM; ++c) part[(g * kKmRows + r) * KM + c] = d2[c];
-    }
-    __syncthreads();
-    if (g == 0 && r < nb) {
-      int best = 0;
-      float bd = 0.f;
-#pragma unroll
-      for (int c = 0; c < KM; ++c) {
-        float d = part[r * KM + c];
-#pragma unroll
-        for (int gg = 1; gg < 4; ++gg) d += part[(gg * kKmRows + r) * KM + c];
-        if (c == 0 || d < bd) {
-          bd = d;
-          best = c;
-        }
-      }
-      sassign[r] = best;
-    }
-    __syncthreads();
-    // update: partial member sums of dimension r over one quarter of the queries
-    if (r < D) {
-      float acc[KM];
-      int n[KM];
-#pragma unroll
-      for (int c = 0; c < KM; ++c) {
-        acc[c] = 0.f;
-        n[c] = 0;
-      }
-      const int t1 = min(nb, (g + 1) * (kKmRows / 4));
-      for (int t = g * (kKmRows / 4); t < t1; ++t) {
-        const int as = sassign[t];
-        const float x = sq[t * QS + r];
+      for (int i = 0; i < 8; ++i) {
 #pragma unroll
         for (int c = 0; c < KM; ++c) {
-          if (as == c) {
-            acc[c] += x;
-            ++n[c];
+          const float4 nc = *reinterpret_cast<const float4*>(&sm.negc[c * D + 32 * g + 4 * i]);
+          const float2 n0 = make_float2(nc.x, nc.y), n1 = make_float2(nc.z, nc.w);
+#pragma unroll
+          for (int qi = 0; qi < 2; ++qi) {
+            const float2 t0 = __fadd2_rn(x[qi][2 * i], n0);
+            acc[qi][c] = __ffma2_rn(t0, t0, acc[qi][c]);
+            const float2 t1 = __fadd2_rn(x[qi][2 * i + 1], n1);
+            acc[qi][c] = __ffma2_rn(t1, t1, acc[qi][c]);
           }
         }
       }
 #pragma unroll
-      for (int c = 0; c < KM; ++c) part[(g * KM + c) * D + r] = acc[c];
-      if (r == 0) {
+      for (int qi = 0; qi < 2; ++qi)
 #pragma unroll
-        for (int c = 0; c < KM; ++c) pcount[g * KM + c] = n[c];
+        for (int c = 0; c < KM; ++c)
+          sm.part[(g * KM + c) * kKmRows + p + 64 * qi] = acc[qi][c].x + acc[qi][c].y;
+    }
+    __syncthreads();
+    // ---- argmin and counting sort (warps 0-3: thread r = query r)
+    int best = -1, rank = 0;
+    if (tid < kKmRows) {
+      const int r = tid;
+      if (r < nb) {
+        float bd = 0.f;
+#pragma unroll
+        for (int c = 0; c < KM; ++c) {
+          float d = sm.part[c * kKmRows + r];
+#pragma unroll
+          for (int gg = 1; gg < 4; ++gg) d += sm.part[(gg * KM + c) * kKmRows + r];
+          if (c == 0 || d < bd) {
+            bd = d;
+            best = c;
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < KM; ++c) {
+        const unsigned bal = __ballot_sync(0xffffffffu, best == c);
+        if (best == c) rank = __popc(bal & ((1u << lane) - 1u));
+        if (lane == 0) sm.wcount[warp][c] = __popc(bal);
       }
     }
     __syncthreads();
-    if (g == 0 && r < D) {
+    if (tid < kKmRows) {
+      if (best >= 0) {
+        int pos = rank;
+        for (int c = 0; c < best; ++c)
+#pragma unroll
+          for (int w = 0; w < 4; ++w) pos += sm.wcount[w][c];
+        for (int w = 0; w < warp; ++w) pos += sm.wcount[w][best];
+        sm.perm[pos] = tid;
+      }
+      if (tid <= KM) {
+        int s0 = 0;
+        for (int c = 0; c < tid; ++c)
+#pragma unroll
+          for (int w = 0; w < 4; ++w) s0 += sm.wcount[w][c];
+        sm.start[tid] = s0;
+      }
+    }
+    __syncthreads();
+    // ---- update: member sums of dimension pair j over sorted quarter s
+    {
+      const int s = tid >> 6, j = tid & 63;
+      const int lo = (s * nb) >> 2, hi = ((s + 1) * nb) >> 2;
 #pragma unroll
       for (int c = 0; c < KM; ++c) {
-        const int n = pcount[c] + pcount[KM + c] + pcount[2 * KM + c] + pcount[3 * KM + c];
-        float acc = part[c * D + r];
+        const int a = max(lo, sm.start[c]), b = min(hi, sm.start[c + 1]);
+        float2 acc = make_float2(0.f, 0.f);
+        for (int t = a; t < b; ++t) {
+          const uint32_t w =
+              *reinterpret_cast<const uint32_t*>(&sm.q[sm.perm[t] * kKmRowPitch + 2 * j]);
+          acc = __fadd2_rn(acc, make_float2(__uint_as_float(w << 16),
+                                            __uint_as_float(w & 0xffff0000u)));
+        }
+        *reinterpret_cast<float2*>(&sm.part[(s * KM + c) * D + 2 * j]) = acc;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < KM * D; i += kKmThreads) {
+      const int c = i / D, col = i - c * D;
+      const int n = sm.start[c + 1] - sm.start[c];
+      if (n > 0) {
+        float acc = sm.part[c * D + col];
 #pragma unroll
-        for (int gg = 1; gg < 4; ++gg) acc += part[(gg * KM + c) * D + r];
-        if (n > 0) sc[c * D + r] = acc / static_cast<float>(n);
-        if (r == 0) scount[c] = n;
+        for (int s = 1; s < 4; ++s) acc += sm.part[(s * KM + c) * D + col];
+        sm.negc[i] = -(acc / static_cast<float>(n));
       }
     }
     __syncthreads();
   }
   float* co = cent + static_cast<size_t>(row) * KM * D;
-  for (int i = threadIdx.x; i < KM * D; i += kKmThreads) co[i] = sc[i];
-  if (threadIdx.x < KM) {
-    const int n = iters > 0 ? scount[threadIdx.x] : 0;
-    wts[static_cast<size_t>(row) * KM + threadIdx.x] =
-        static_cast<float>(n) / static_cast<float>(nb);
+  for (int i = tid; i < KM * D; i += kKmThreads) co[i] = -sm.negc[i];
+  if (tid < KM) {
+    const int n = iters > 0 ? sm.start[tid + 1] - sm.start[tid] : 0;
+    wts[static_cast<size_t>(row) * KM + tid] = static_cast<float>(n) / static_cast<float>(nb);
   }
 }
 
@@ -323,16 +376,14 @@ __global__ void __launch_bounds__(kSipThreads) sip_sample_kernel(
   }
 }
 
-template <int D, int KM>
+template <int KM>
 cudaError_t launch_kmeans_t(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
                             int B, int iters, cudaStream_t s) {
   const int nqb = (N + B - 1) / B;
-  const size_t km_smem =
-      sizeof(float) * (static_cast<size_t>(kKmRows) * (D + 1) + KM * D + 4 * kKmRows * KM) +
-      sizeof(int) * (kKmRows + 4 * KM);
-  cudaError_t e = set_dyn_smem<kmeans_kernel<D, KM>>(static_cast<int>(km_smem));
+  const int smem = static_cast<int>(sizeof(KmSmem<KM>));
+  cudaError_t e = set_dyn_smem<kmeans_kernel<KM>>(smem);
   if (e != cudaSuccess) return e;
-  kmeans_kernel<D, KM><<<heads * nqb, kKmThreads, km_smem, s>>>(q, N, B, nqb, iters, cent, wts);
+  kmeans_kernel<KM><<<heads * nqb, kKmThreads, smem, s>>>(q, N, B, nqb, iters, cent, wts);
   return cudaGetLastError();
 }
 
@@ -342,16 +393,13 @@ int ibcs_max_subblocks() { return static_cast<int>((200 * 1024) / (sizeof(float)
 
 cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
                           int d, int B, int km_k, int iters, cudaStream_t s) {
-#define STA_KM_CASE(DD, KK) \
-  if (d == DD && km_k == KK) return launch_kmeans_t<DD, KK>(q, cent, wts, heads, N, B, iters, s);
-  STA_KM_CASE(128, 4)
-  STA_KM_CASE(128, 2)
-  STA_KM_CASE(128, 1)
-  STA_KM_CASE(128, 8)
-  STA_KM_CASE(64, 4)
-  STA_KM_CASE(64, 2)
-  STA_KM_CASE(64, 1)
-  STA_KM_CASE(64, 8)
+#define STA_KM_CASE(KK) \
+  if (km_k == KK) return launch_kmeans_t<KK>(q, cent, wts, heads, N, B, iters, s);
+  if (d != 128 || B < 1 || B > kKmRows) return cudaErrorInvalidValue;
+  STA_KM_CASE(4)
+  STA_KM_CASE(2)
+  STA_KM_CASE(1)
+  STA_KM_CASE(8)
 #undef STA_KM_CASE
   return cudaErrorInvalidValue;
 }

@@ -127,3 +127,17 @@ def test_fraction_one_keeps_everything_unweighted(cuda_ok):
     torch.cuda.synchronize()
     ref = np.concatenate([dense_rows(q[0], k[0], v[0], qb, 128) for qb in range(4)])
     assert_close_attn(o[0].float().cpu().numpy(), ref, "frac=1 vs dense")
+
+
+@pytest.mark.parametrize("k,block_q", [(1, 128), (2, 128), (8, 128), (4, 64)])
+def test_ibcs_centroid_counts_and_query_blocks(cuda_ok, k, block_q):
+    """Other centroid counts and a 64-query block (ragged last block)."""
+    w = workload("ab_sampled", heads=2, F=3, H=10, W=13, block_q=block_q)   # N = 390
+    w["ibcs"]["k"] = k
+    w["ibcs"]["sample_frac"] = 0.25
+    q, k_, _ = make_qkv(w)
+    L = _gpu_select(w, q.cuda(), k_.cuda())
+    checked, skipped, near = _check_rows(w, L, q, k_, (0, 1), None)
+    # k = 8 on the 6-query last block starts two centroids on the same query:
+    # an exact tie (margin 0), so that row of each head is not compared
+    assert checked >= 4 and skipped <= 2 and near <= 2
