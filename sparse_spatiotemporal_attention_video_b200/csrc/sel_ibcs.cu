@@ -236,24 +236,6 @@ __global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 1 : 2) kmeans_kernel(
 constexpr int kSipThreads = 256;
 constexpr int kSipWarps = kSipThreads / 32;
 
-// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
-// easy as 1, 2, 3", SC'11): ten rounds of two 32x32->64-bit multiplies whose
-// high halves are XOR-ed with the other two counter words and the key, with
-// the key bumped by two Weyl constants between rounds.
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
-  constexpr uint32_t kM0 = 0xD2511F53u, kM1 = 0xCD9E8D57u;
-  constexpr uint32_t kW0 = 0x9E3779B9u, kW1 = 0xBB67AE85u;
-#pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    const uint32_t hi0 = __umulhi(kM0, c.x), lo0 = kM0 * c.x;
-    const uint32_t hi1 = __umulhi(kM1, c.z), lo1 = kM1 * c.z;
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
-    k0 += kW0;
-    k1 += kW1;
-  }
-  return c;
-}
-
 __device__ __forceinline__ double block_sum_d(double v, double* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -288,88 +270,133 @@ __device__ __forceinline__ int block_sum_i(int v, int* red, int& excl) {
   return tot;
 }
 
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
+// easy as 1, 2, 3", SC'11): ten rounds of two 32x32->64-bit multiplies whose
+// high halves are XOR-ed with the other two counter words and the key, with
+// the key bumped by two Weyl constants between rounds.  Two counter blocks
+// are advanced in lockstep (independent chains: the multiplies of one overlap
+// the dependent steps of the other).
+__device__ __forceinline__ void philox4x32_10_x2(uint4& a, uint4& b, uint32_t k0, uint32_t k1) {
+  constexpr uint32_t kM0 = 0xD2511F53u, kM1 = 0xCD9E8D57u;
+  constexpr uint32_t kW0 = 0x9E3779B9u, kW1 = 0xBB67AE85u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t ah0 = __umulhi(kM0, a.x), al0 = kM0 * a.x;
+    const uint32_t ah1 = __umulhi(kM1, a.z), al1 = kM1 * a.z;
+    const uint32_t bh0 = __umulhi(kM0, b.x), bl0 = kM0 * b.x;
+    const uint32_t bh1 = __umulhi(kM1, b.z), bl1 = kM1 * b.z;
+    a = make_uint4(ah1 ^ a.y ^ k0, al1, ah0 ^ a.w ^ k1, al0);
+    b = make_uint4(bh1 ^ b.y ^ k0, bl1, bh0 ^ b.w ^ k1, bl0);
+    k0 += kW0;
+    k1 += kW1;
+  }
+}
+
+// One CTA per (head, query block) row of p.  Shared memory: p of the row
+// (ld = n_sub rounded up to 4 floats) and one flag byte per sub-block
+// (bit 0 capped, bit 1 kept).
+//  - Water filling: each round caps every uncapped j with lambda p_j >= 1
+//    and, in the same pass, sums (fp64) the p of the sub-blocks that stay
+//    uncapped, which is the next round's denominator.
+//  - Draws: thread t takes the Philox groups t, t + T, ... two at a time and
+//    sets the kept bit where u_j < pi_j; pi_j = 1 for capped j, else
+//    min(1, lambda p_j) in fp64.
+//  - Output: thread t owns a contiguous chunk of sub-blocks (a multiple of 4),
+//    counts its kept bits, and an exclusive block scan places its ids in
+//    ascending order, with logw = -ln pi.
 __global__ void __launch_bounds__(kSipThreads) sip_sample_kernel(
     const float* __restrict__ p, int n_sub, int m, uint32_t seed_lo, uint32_t seed_hi,
     int32_t* __restrict__ idx, float* __restrict__ logw, int32_t* __restrict__ cnt, int cap,
     int32_t* required_cap, int32_t* dev_status) {
-  extern __shared__ float sip_smem[];
-  float* sp = sip_smem;                                    // [n_sub]
-  uint8_t* capped = reinterpret_cast<uint8_t*>(sp + n_sub);  // [n_sub]
+  extern __shared__ __align__(16) float sip_smem[];
+  const int ld = (n_sub + 3) & ~3;
+  float* sp = sip_smem;                                          // [ld]
+  uint8_t* flag = reinterpret_cast<uint8_t*>(sp + ld);           // [ld]
   __shared__ double redd[kSipWarps];
   __shared__ int redi[kSipWarps];
+  const int tid = threadIdx.x;
   const int row = blockIdx.x;  // head * nqb + qb
-  const float* pr = p + static_cast<size_t>(row) * ((n_sub + 3) & ~3);  // 16-byte rows
-  for (int j = threadIdx.x; j < n_sub; j += kSipThreads) {
-    sp[j] = __ldcs(pr + j);
-    capped[j] = 0;
+  const float4* pr = reinterpret_cast<const float4*>(p + static_cast<size_t>(row) * ld);
+  double part = 0.0;
+  for (int i = tid; i < ld / 4; i += kSipThreads) {
+    const float4 v = __ldcs(pr + i);  // padding columns hold 0
+    reinterpret_cast<float4*>(sp)[i] = v;
+    reinterpret_cast<uint32_t*>(flag)[i] = 0u;
+    part += (static_cast<double>(v.x) + static_cast<double>(v.y)) +
+            (static_cast<double>(v.z) + static_cast<double>(v.w));
   }
-  __syncthreads();
+  double rest = block_sum_d(part, redd);  // its barriers also publish sp / flag
   // water filling
   int ncap = 0;
   double lam = 0.0;
-  for (int iter = 0; iter <= n_sub; ++iter) {
-    double part = 0.0;
-    for (int j = threadIdx.x; j < n_sub; j += kSipThreads)
-      if (!capped[j]) part += static_cast<double>(sp[j]);
-    const double rest = block_sum_d(part, redd);
-    if (!(rest > 0.0)) break;
+  for (int round = 0; round <= n_sub && rest > 0.0; ++round) {
     lam = static_cast<double>(m - ncap) / rest;
     int newc = 0;
-    for (int j = threadIdx.x; j < n_sub; j += kSipThreads) {
-      if (!capped[j] && lam * static_cast<double>(sp[j]) >= 1.0) {
-        capped[j] = 1;
-        ++newc;
+    part = 0.0;
+    for (int j = tid; j < n_sub; j += kSipThreads) {
+      if (!flag[j]) {
+        const double pj = static_cast<double>(sp[j]);
+        if (lam * pj >= 1.0) {
+          flag[j] = 1;
+          ++newc;
+        } else {
+          part += pj;
+        }
       }
     }
     int dummy;
     const int tot = block_sum_i(newc, redi, dummy);
     if (tot == 0) break;
     ncap += tot;
+    rest = block_sum_d(part, redd);
   }
-  // Poisson sampling over a contiguous chunk per thread, ascending output
-  const int chunk = (n_sub + kSipThreads - 1) / kSipThreads;
-  const int j_lo = min(n_sub, threadIdx.x * chunk);
-  const int j_hi = min(n_sub, j_lo + chunk);
   auto pi_of = [&](int j) -> double {
-    if (capped[j]) return 1.0;
+    if (flag[j] & 1) return 1.0;
     return fmin(1.0, lam * static_cast<double>(sp[j]));
   };
-  auto keep_of = [&](int j, uint4& words, int& group) -> bool {
-    if ((j >> 2) != group) {
-      group = j >> 2;
-      words = philox4x32_10(make_uint4(static_cast<uint32_t>(group), 0u,
-                                       static_cast<uint32_t>(row), 0u),
-                            seed_lo, seed_hi);
+  // draws
+  const int n_grp = ld / 4;
+  const uint32_t ctr = static_cast<uint32_t>(row);
+  auto mark = [&](int g, uint4 w) {
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * g + e;
+      if (j < n_sub && static_cast<double>(x[e] >> 8) * (1.0 / 16777216.0) < pi_of(j))
+        flag[j] |= 2;
     }
-    const uint32_t x = (j & 3) == 0 ? words.x : (j & 3) == 1 ? words.y : (j & 3) == 2 ? words.z : words.w;
-    const double u = static_cast<double>(x >> 8) * (1.0 / 16777216.0);
-    return u < pi_of(j);
   };
-  int mine = 0;
-  {
-    uint4 w = make_uint4(0, 0, 0, 0);
-    int g = -1;
-    for (int j = j_lo; j < j_hi; ++j) mine += keep_of(j, w, g) ? 1 : 0;
+  for (int g = tid; g < n_grp; g += 2 * kSipThreads) {
+    const int g2 = g + kSipThreads;
+    uint4 a = make_uint4(static_cast<uint32_t>(g), 0u, ctr, 0u);
+    uint4 b = make_uint4(static_cast<uint32_t>(g2), 0u, ctr, 0u);
+    philox4x32_10_x2(a, b, seed_lo, seed_hi);
+    mark(g, a);
+    if (g2 < n_grp) mark(g2, b);
   }
+  __syncthreads();
+  // ascending output
+  const int chunk = ((n_grp + kSipThreads - 1) / kSipThreads) * 4;
+  const int j_lo = min(ld, tid * chunk);
+  const int j_hi = min(ld, j_lo + chunk);
+  int mine = 0;
+  for (int j = j_lo; j < j_hi; j += 4)
+    mine += __popc(reinterpret_cast<const uint32_t*>(flag)[j >> 2] & 0x02020202u);
   int before;
   const int total = block_sum_i(mine, redi, before);
-  {
-    uint4 w = make_uint4(0, 0, 0, 0);
-    int g = -1;
-    int pos = before;
-    int32_t* out = idx + static_cast<size_t>(row) * cap;
-    float* lw = logw ? logw + static_cast<size_t>(row) * cap : nullptr;
-    for (int j = j_lo; j < j_hi; ++j) {
-      if (keep_of(j, w, g)) {
-        if (pos < cap) {
-          out[pos] = j;
-          if (lw) lw[pos] = static_cast<float>(-log(pi_of(j)));
-        }
-        ++pos;
+  int pos = before;
+  int32_t* out = idx + static_cast<size_t>(row) * cap;
+  float* lw = logw ? logw + static_cast<size_t>(row) * cap : nullptr;
+  for (int j = j_lo; j < j_hi; ++j) {
+    if (flag[j] & 2) {
+      if (pos < cap) {
+        out[pos] = j;
+        if (lw) lw[pos] = static_cast<float>(-log(pi_of(j)));
       }
+      ++pos;
     }
   }
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     cnt[row] = min(total, cap);
     if (required_cap) atomicMax(required_cap, total);
     if (total > cap) raise_status(dev_status, STA_DEV_CAPACITY);
@@ -407,7 +434,7 @@ cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int h
 cudaError_t launch_sip_sample(const float* p, int rows, int n_sub, int m, uint64_t seed,
                               int32_t* idx, float* logw, int32_t* cnt, int cap,
                               int32_t* required_cap, int32_t* dev_status, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(n_sub) * (sizeof(float) + 1);
+  const size_t smem = static_cast<size_t>((n_sub + 3) & ~3) * (sizeof(float) + 1);
   cudaError_t e = set_dyn_smem<sip_sample_kernel>(static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   sip_sample_kernel<<<rows, kSipThreads, smem, s>>>(
