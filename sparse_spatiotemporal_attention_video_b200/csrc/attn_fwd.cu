@@ -460,6 +460,9 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       wq = rem - hq * a.W;
     }
     const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
+    const bool weighted = !dense_like && a.logw != nullptr;
+    const int n_full = a.N / UNIT;  // units whose keys all lie below N
+    const int n_units = (a.N + UNIT - 1) / UNIT;
     float m_run = -INFINITY, l_run = 0.f;
     HalfRaw<UNIT> raw_next;
     if (!dense_like) load_half_raw<UNIT>(a, I, 0, J, raw_next);
@@ -467,18 +470,21 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       const uint32_t gg = g + t;
       const uint32_t sb = gg & 1;
       const uint32_t tS = tmem + lane_off + sb * 128;
-      HalfInfo<kTileK> td;
-      HalfInfo<UNIT> ti;
-      bool simple;  // no masked column, no weight, no window
+      // Only the raw entries stay live across the tile; the per-slot masks
+      // are derived from them on the (rare) masked path.
+      HalfRaw<UNIT> raw = {};
+      bool full;  // every column of the group's half is a valid key
       if (dense_like) {
-        load_half_info<kTileK>(a, I, t, J, inv_scale, td);  // geometry only, no loads
-        simple = td.full;
+        full = (t * kTileK + J * 64 + 64 <= a.N);
       } else {
-        const HalfRaw<UNIT> raw = raw_next;
-        half_info_from_raw<UNIT>(a, I, J, inv_scale, raw, ti);
-        simple = ti.full && !ti.bias && !window;
+        raw = raw_next;
+        full = true;
+#pragma unroll
+        for (int q = 0; q < HalfInfo<UNIT>::SLOTS; ++q)
+          full = full && (static_cast<unsigned>(raw.u[q]) < static_cast<unsigned>(n_full));
         load_half_raw<UNIT>(a, I, t + 1, J, raw_next);  // next tile's entries
       }
+      const bool simple = full && !weighted && !window;  // no mask, no weight
       if (!mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit)) {
         ok = false;
         break;
@@ -486,15 +492,26 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       tc_fence_after();
       float x[64];
       load_cols64(tS + J * 64, x);
-      if (!simple) {
-        if (dense_like) mask_half<kTileK>(x, td, false, a, 0, 0, 0);
-        else mask_half<UNIT>(x, ti, window, a, fq, hq, wq);
+      if (!full || window) {
+        if (dense_like) {
+          HalfInfo<kTileK> td;
+          load_half_info<kTileK>(a, I, t, J, inv_scale, td);  // geometry only, no loads
+          mask_half<kTileK>(x, td, false, a, 0, 0, 0);
+        } else {
+          HalfInfo<UNIT> ti;
+          half_info_from_raw<UNIT>(a, I, J, inv_scale, raw, ti);
+          mask_half<UNIT>(x, ti, window, a, fq, hq, wq);
+        }
       }
-      // per-slot log-weights (raw logit units), 0 without weights
+      // per-slot log-weights (raw logit units), 0 without weights (a masked
+      // slot's value does not matter: its logits are -inf)
       constexpr int SW = HalfInfo<UNIT>::W, NS = HalfInfo<UNIT>::SLOTS;
       float bias[NS];
 #pragma unroll
-      for (int q = 0; q < NS; ++q) bias[q] = (!dense_like && ti.bias) ? ti.braw[q] : 0.f;
+      for (int q = 0; q < NS; ++q)
+        bias[q] = (weighted && static_cast<unsigned>(raw.u[q]) < static_cast<unsigned>(n_units))
+                      ? raw.lw[q] * inv_scale
+                      : 0.f;
       float ms[NS];
       slot_max<SW>(x, ms);
       float mraw = ms[0] + bias[0];
@@ -595,15 +612,15 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
           float4* op = reinterpret_cast<float4*>(static_cast<float*>(a.o) + gcol);
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            op[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+            __stcs(op + i, make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
         } else {
           uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.o) + gcol);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
-            op[i] = make_uint4(pack_bf16x2(o[8 * i], o[8 * i + 1]),
-                               pack_bf16x2(o[8 * i + 2], o[8 * i + 3]),
-                               pack_bf16x2(o[8 * i + 4], o[8 * i + 5]),
-                               pack_bf16x2(o[8 * i + 6], o[8 * i + 7]));
+            __stcs(op + i, make_uint4(pack_bf16x2(o[8 * i], o[8 * i + 1]),
+                                      pack_bf16x2(o[8 * i + 2], o[8 * i + 3]),
+                                      pack_bf16x2(o[8 * i + 4], o[8 * i + 5]),
+                                      pack_bf16x2(o[8 * i + 6], o[8 * i + 7])));
         }
       }
     }
@@ -690,6 +707,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // K/V tiles are read by every query block of a head: keep them in L2
+    // ahead of the Q tiles, which are read once.
+    const uint64_t pol_kv = l2_policy_evict_last();
+    const uint64_t pol_q = l2_policy_evict_first();
     uint32_t kt = 0, vt = 0, qn = 0;
     for (int it = blockIdx.x; it < a.n_items; it += gridDim.x) {
       if (*abort) break;
@@ -725,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(q_full, L::TILE_BYTES);
 #pragma unroll
         for (int h = 0; h < L::DH; ++h)
-          tma_load_3d(sQ + h * kHalfBytes, &tm_q, q_full, h * 64, I.q_start, I.head);
+          tma_load_3d_hint(sQ + h * kHalfBytes, &tm_q, q_full, h * 64, I.q_start, I.head, pol_q);
       }
       ++qn;
       const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
@@ -753,8 +774,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive_expect_tx(k_full + st, L::TILE_BYTES);
           __syncwarp();
           if (lane < nops)
-            tma_load_3d(sK + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mk,
-                        k_full + st, h * 64, u * unit, I.head);
+            tma_load_3d_hint(sK + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mk,
+                             k_full + st, h * 64, u * unit, I.head, pol_kv);
           ++kt;
         }
         // V
@@ -766,8 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive_expect_tx(v_full + st, L::TILE_BYTES);
           __syncwarp();
           if (lane < nops)
-            tma_load_3d(sV + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mv,
-                        v_full + st, h * 64, u * unit, I.head);
+            tma_load_3d_hint(sV + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mv,
+                             v_full + st, h * 64, u * unit, I.head, pol_kv);
           ++vt;
         }
       }
