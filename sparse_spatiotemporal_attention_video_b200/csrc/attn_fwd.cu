@@ -630,14 +630,40 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
   if (!ok) fail(abort, a.dev_status);
 }
 
+// Slot s of a K or V tile in the interleaved layout ([8-row group][half]
+// [8 rows][128 B]): one copy through the five-dimensional view when the
+// unit lies in whole 8-row groups below N & ~7 (u < n_il), else 8-row copies
+// per half through the three-dimensional map, which zero-fills rows past N.
+template <int UNIT>
+__device__ __forceinline__ void load_unit_il(uint8_t* tile, const CUtensorMap* m_il,
+                                             const CUtensorMap* m8, uint64_t* bar, int s, int u,
+                                             int n_il, int head, uint64_t pol) {
+  constexpr int G = UNIT / 8;  // 8-row groups per unit
+  uint8_t* dst = tile + s * G * 2048;
+  if (u < n_il) {
+    tma_load_5d_hint(dst, m_il, bar, 0, 0, 0, u * G, head, pol);
+  } else {
+#pragma unroll
+    for (int j = 0; j < G; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        tma_load_3d_hint(dst + j * 2048 + h * 1024, m8, bar, h * 64, u * UNIT + 8 * j, head, pol);
+  }
+}
+
 template <int D, int KS, int VS, int UNIT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k_u,
                     const __grid_constant__ CUtensorMap tm_v_u,
                     const __grid_constant__ CUtensorMap tm_k_f,
-                    const __grid_constant__ CUtensorMap tm_v_f) {
+                    const __grid_constant__ CUtensorMap tm_v_f,
+                    const __grid_constant__ CUtensorMap tm_k_il,
+                    const __grid_constant__ CUtensorMap tm_v_il) {
   using L = Layout<D, KS, VS>;
+  // d = 128 with units shorter than 64 keys: list tiles use the interleaved
+  // layout [8-row group][half][8 rows][128 B] (one TMA copy per unit)
+  constexpr bool kInterleaved = (D == 128 && UNIT < 64);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -692,6 +718,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_v_u);
     tma_prefetch_desc(&tm_k_f);
     tma_prefetch_desc(&tm_v_f);
+    if (kInterleaved) {
+      tma_prefetch_desc(&tm_k_il);
+      tma_prefetch_desc(&tm_v_il);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -753,11 +783,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const CUtensorMap* mk = dense_like ? &tm_k_f : &tm_k_u;
       const CUtensorMap* mv = dense_like ? &tm_v_f : &tm_v_u;
       const int unit = I.unit;
-      const int nops = I.upt * L::DH;
+      const bool il = kInterleaved && !dense_like;
+      const int nops = il ? I.upt : I.upt * L::DH;
+      const int n_il = (a.N & ~7) / UNIT;  // units the interleaved view covers
       for (int t = 0; t < I.ntiles; ++t) {
-        // one lane per (slot, half) copy
+        // one lane per (slot, half) copy, or per slot in the interleaved layout
         int u = 0;
-        const int s = lane / L::DH, h = lane % L::DH;
+        const int s = il ? lane : lane / L::DH, h = il ? 0 : lane % L::DH;
         if (lane < nops) {
           int nv;
           float lw;
@@ -773,9 +805,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           if (lane == 0) mbar_arrive_expect_tx(k_full + st, L::TILE_BYTES);
           __syncwarp();
-          if (lane < nops)
+          if (il) {
+            if (lane < nops)
+              load_unit_il<UNIT>(sK + st * L::TILE_BYTES, &tm_k_il, mk, k_full + st, s, u, n_il,
+                           I.head, pol_kv);
+          } else if (lane < nops) {
             tma_load_3d_hint(sK + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mk,
                              k_full + st, h * 64, u * unit, I.head, pol_kv);
+          }
           ++kt;
         }
         // V
@@ -786,9 +823,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           if (lane == 0) mbar_arrive_expect_tx(v_full + st, L::TILE_BYTES);
           __syncwarp();
-          if (lane < nops)
+          if (il) {
+            if (lane < nops)
+              load_unit_il<UNIT>(sV + st * L::TILE_BYTES, &tm_v_il, mv, v_full + st, s, u, n_il,
+                           I.head, pol_kv);
+          } else if (lane < nops) {
             tma_load_3d_hint(sV + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mv,
                              v_full + st, h * 64, u * unit, I.head, pol_kv);
+          }
           ++vt;
         }
       }
@@ -818,6 +860,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // groups have read them out (o_free).
       bool first = true;
       bool wait_free = false;
+      // K/V tiles of the current item are in the interleaved layout: 8-row
+      // groups 2048 bytes apart, halves 1024 apart (else 1024 and 16384)
+      bool il = false;
       auto issue_pv = [&](uint32_t gg) -> bool {
         const uint32_t sb = gg & 1;
         if (!mbar_wait(p_full + sb, (gg >> 1) & 1, abort, limit)) return false;
@@ -833,7 +878,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vbase = aV + st * L::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < kTileK / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024);
+          // V is MN-major: LBO steps between the two 64-column halves, SBO
+          // between the two 8-key groups of the 16-key step
+          const uint64_t bdesc = il ? smem_desc_sw128(vbase + kk * 4096, 1024, 2048)
+                                    : smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024);
           // keys 0..63 (softmax group 0): P in columns 0..31, into O_0;
           // keys 64..127 (group 1): P in columns 64..95, into O_1
           const uint32_t pa = tS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
@@ -857,6 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         first = true;
         wait_free = qn > 0;
+        il = kInterleaved && (I.kind == kItemList || I.kind == kItemLocal);
         for (int t = 0; t < I.ntiles; ++t) {
           const int st = kt % KS;
           if (!mbar_wait(k_full + st, (kt / KS) & 1, abort, limit)) {
@@ -871,7 +920,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
             const uint64_t adesc = smem_desc_sw128(aQ + off, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(kbase + off, 16, 1024);
+            const uint64_t bdesc =
+                il ? smem_desc_sw128(kbase + (kk >> 2) * 1024 + (kk & 3) * 32, 16, 2048)
+                   : smem_desc_sw128(kbase + off, 16, 1024);
             mma_bf16_ss(tS, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
           }
           mma_commit(k_empty + st);
@@ -922,14 +973,15 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
 template <int D, int KS, int VS, int UNIT>
 cudaError_t launch_t(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tku,
                      const CUtensorMap& tvu, const CUtensorMap& tkf, const CUtensorMap& tvf,
-                     int num_sms, cudaStream_t stream) {
+                     const CUtensorMap& tki, const CUtensorMap& tvi, int num_sms,
+                     cudaStream_t stream) {
   using L = Layout<D, KS, VS>;
   auto kern = attn_fwd_kernel<D, KS, VS, UNIT>;
   cudaError_t e = set_dyn_smem<attn_fwd_kernel<D, KS, VS, UNIT>>(L::ALLOC);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kThreads, L::ALLOC, stream>>>(a, tq, tku, tvu, tkf, tvf);
+  kern<<<grid, kThreads, L::ALLOC, stream>>>(a, tq, tku, tvu, tkf, tvf, tki, tvi);
   return cudaGetLastError();
 }
 
@@ -937,11 +989,13 @@ cudaError_t launch_t(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap
 
 cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tq,
                              const CUtensorMap& tku, const CUtensorMap& tvu,
-                             const CUtensorMap& tkf, const CUtensorMap& tvf, int num_sms,
+                             const CUtensorMap& tkf, const CUtensorMap& tvf,
+                             const CUtensorMap& tki, const CUtensorMap& tvi, int num_sms,
                              cudaStream_t stream) {
-#define STA_ATTN_CASE(DD, UU)                                                                \
-  if (d == DD && a.unit == UU)                                                               \
-    return launch_t<DD, STA_KSTAGES, STA_VSTAGES, UU>(a, tq, tku, tvu, tkf, tvf, num_sms, stream);
+#define STA_ATTN_CASE(DD, UU)                                                              \
+  if (d == DD && a.unit == UU)                                                             \
+    return launch_t<DD, STA_KSTAGES, STA_VSTAGES, UU>(a, tq, tku, tvu, tkf, tvf, tki, tvi, \
+                                                      num_sms, stream);
   STA_ATTN_CASE(128, 128)
   STA_ATTN_CASE(128, 64)
   STA_ATTN_CASE(128, 32)

@@ -60,10 +60,14 @@ struct AttnArgs {
   int32_t* dev_status;
 };
 
-// Launchers (attn_fwd.cu).
+// Launchers (attn_fwd.cu).  With d = 128 and units shorter than 64 keys the
+// unit maps have 8-row boxes and tm_k_il / tm_v_il are the interleaved
+// five-dimensional views (see interleaved_unit_map); otherwise those two are
+// unused.
 cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tm_q,
                              const CUtensorMap& tm_k_unit, const CUtensorMap& tm_v_unit,
                              const CUtensorMap& tm_k_full, const CUtensorMap& tm_v_full,
+                             const CUtensorMap& tm_k_il, const CUtensorMap& tm_v_il,
                              int num_sms, cudaStream_t stream);
 cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
 

@@ -59,6 +59,27 @@ bool make_map(CUtensorMap* m, const void* base, int d, int N, int heads, int box
   return r == CUDA_SUCCESS;
 }
 
+// Five-dimensional view of a [heads][N][128] bf16 tensor for loading one
+// key/value unit of `unit` rows (both 64-column halves) in a single TMA copy:
+// dims (64 columns, 8 rows, 2 halves, N/8 row groups, heads) with byte
+// strides (256, 128, 2048, N*256) and box (64, 8, 2, unit/8, 1).  The box
+// lands in shared memory as [row group][half][8 rows][128 B], each 1 KB
+// block one 128-byte-swizzle atom.  Only row groups below N/8 are in range,
+// so a copy never reads past the head's last row.
+bool interleaved_unit_map(CUtensorMap* m, const void* base, int N, int heads, int unit) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t groups = N >= 8 ? static_cast<cuuint64_t>(N / 8) : 1;
+  cuuint64_t dims[5] = {64, 8, 2, groups, static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[4] = {256, 128, 2048, static_cast<cuuint64_t>(N) * 256};
+  cuuint32_t box[5] = {64, 8, 2, static_cast<cuuint32_t>(unit / 8), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool pow2_unit(int u) { return u == 16 || u == 32 || u == 64 || u == 128; }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -118,21 +139,31 @@ sta_status stage_inputs(const sta_problem* p, const void* q, const void* k, cons
 sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16* qb,
                          const __nv_bfloat16* kb, const __nv_bfloat16* vb, int unit,
                          cudaStream_t stream) {
-  CUtensorMap tq, tku, tvu, tkf, tvf;
+  CUtensorMap tq, tku, tvu, tkf, tvf, tki, tvi;
   const int N = a.N;
+  // d = 128 with units shorter than 64 keys: one interleaved copy per unit,
+  // 8-row boxes for a unit that reaches the last N % 8 rows
+  const bool il = (p->d == 128 && unit < 64);
+  const int unit_box = il ? 8 : unit;
   if (!make_map(&tq, qb, p->d, N, p->heads, kTileQ) ||
-      !make_map(&tku, kb, p->d, N, p->heads, unit) ||
-      !make_map(&tvu, vb, p->d, N, p->heads, unit) ||
+      !make_map(&tku, kb, p->d, N, p->heads, unit_box) ||
+      !make_map(&tvu, vb, p->d, N, p->heads, unit_box) ||
       !make_map(&tkf, kb, p->d, N, p->heads, kTileK) ||
-      !make_map(&tvf, vb, p->d, N, p->heads, kTileK)) {
+      !make_map(&tvf, vb, p->d, N, p->heads, kTileK) ||
+      (il && (!interleaved_unit_map(&tki, kb, N, p->heads, unit) ||
+              !interleaved_unit_map(&tvi, vb, N, p->heads, unit)))) {
     g_last_cuda_error = cudaErrorInvalidValue;
     return STA_ERR_CUDA;
+  }
+  if (!il) {
+    tki = tkf;  // unused
+    tvi = tvf;
   }
   const int sms = num_sms_current();
   if (sms <= 0) return STA_ERR_CUDA;
   a.unit = unit;
   a.q = qb;
-  if (failed(launch_attention(p->d, a, tq, tku, tvu, tkf, tvf, sms, stream)))
+  if (failed(launch_attention(p->d, a, tq, tku, tvu, tkf, tvf, tki, tvi, sms, stream)))
     return STA_ERR_CUDA;
   return STA_OK;
 }
