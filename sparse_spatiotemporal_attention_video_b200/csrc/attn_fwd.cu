@@ -12,7 +12,11 @@
 //               tile, of the listed key/value units (kv_unit rows each,
 //               128-byte swizzle) into a K ring and a V ring; gathered query
 //               rows (routed items) are copied by the warp and swizzled by
-//               hand.
+//               hand.  With d = 128, a 16-key unit is one copy of both
+//               halves through a five-dimensional view, and its tile is laid
+//               out [8-row group][half][8 rows][128 B]: a 128-key tile then
+//               takes 8 copies per operand instead of 16 of 2 KB, which the
+//               copy engine serves too slowly to keep the tensor core busy.
 //   warp 1      MMA issuer (one thread): S = Q K^T of tile t into TMEM S
 //               buffer t%2 (tcgen05.mma, M=128 N=128 K=16 steps, both
 //               operands K-major in shared memory), then O_0 += P[:, 0:64]
@@ -661,9 +665,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_k_il,
                     const __grid_constant__ CUtensorMap tm_v_il) {
   using L = Layout<D, KS, VS>;
-  // d = 128 with units shorter than 64 keys: list tiles use the interleaved
-  // layout [8-row group][half][8 rows][128 B] (one TMA copy per unit)
-  constexpr bool kInterleaved = (D == 128 && UNIT < 64);
+  // d = 128 with 16-key units: list tiles use the interleaved layout
+  // [8-row group][half][8 rows][128 B], one TMA copy per unit (two 2 KB
+  // copies per unit, one per half, measured 18% slower; from 32 keys up the
+  // per-half copies are the faster form)
+  constexpr bool kInterleaved = (D == 128 && UNIT < 32);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));

@@ -60,7 +60,7 @@ struct AttnArgs {
   int32_t* dev_status;
 };
 
-// Launchers (attn_fwd.cu).  With d = 128 and units shorter than 64 keys the
+// Launchers (attn_fwd.cu).  With d = 128 and 16-key units the
 // unit maps have 8-row boxes and tm_k_il / tm_v_il are the interleaved
 // five-dimensional views (see interleaved_unit_map); otherwise those two are
 // unused.

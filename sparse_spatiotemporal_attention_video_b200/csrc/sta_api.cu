@@ -141,9 +141,9 @@ sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16*
                          cudaStream_t stream) {
   CUtensorMap tq, tku, tvu, tkf, tvf, tki, tvi;
   const int N = a.N;
-  // d = 128 with units shorter than 64 keys: one interleaved copy per unit,
+  // d = 128 with 16-key units: one interleaved copy per unit,
   // 8-row boxes for a unit that reaches the last N % 8 rows
-  const bool il = (p->d == 128 && unit < 64);
+  const bool il = (p->d == 128 && unit < 32);
   const int unit_box = il ? 8 : unit;
   if (!make_map(&tq, qb, p->d, N, p->heads, kTileQ) ||
       !make_map(&tku, kb, p->d, N, p->heads, unit_box) ||
