@@ -46,8 +46,8 @@ L2_FLUSH_BYTES = 256 * 1024 * 1024
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of attn_fwd.cu, first 16 hex).
-NCU_TRAFFIC = {"source_sha": "b2ef84dd709f5501", "workload": "wan_radial",
-               "bytes_per_launch": 304179200 + 88765952}
+NCU_TRAFFIC = {"source_sha": "63af3aaa9acbc04d", "workload": "wan_radial",
+               "bytes_per_launch": 303490304 + 85012480}
 
 
 def parse(argv=None):
