@@ -56,8 +56,10 @@
 namespace sta {
 namespace {
 
-// Warp 0 producer, warp 1 MMA issuer, warps 2-9 two softmax groups.
-constexpr int kThreads = 320;
+// Warp 0 Q/K producer, warp 1 MMA issuer, warps 2-9 two softmax groups,
+// warp 10 V producer.
+constexpr int kWarpV = 10;
+constexpr int kThreads = 352;
 constexpr int kHalfBytes = 128 * 128;  // 128 rows x 128 bytes: one 64-column half of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -73,6 +75,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 #define STA_RESCALE_THRESHOLD 8.0f
 #endif
 constexpr float kRescaleThreshold = STA_RESCALE_THRESHOLD;
+// Speculative row maximum (see softmax_role); 0 finds each tile's maximum
+// before its exponentials.
+#ifndef STA_SPEC_MAX
+#define STA_SPEC_MAX 0
+#endif
+// K/V ring depths: two stages each, one per S buffer, so that a ring slot
+// is free exactly when the MMA that read it has been committed (see the
+// producers); deeper rings measured no faster.
 #ifndef STA_KSTAGES
 #define STA_KSTAGES 2
 #endif
@@ -88,13 +98,11 @@ struct Layout {
   static constexpr int OFF_K = OFF_Q + TILE_BYTES;
   static constexpr int OFF_V = OFF_K + KS * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + VS * TILE_BYTES;
-  // barriers: q_full, q_empty, k_full[KS], k_empty[KS], v_full[VS],
-  // v_empty[VS], s_full[2], p_full[2], o_done[2], o_free, mma_done, and the
+  // barriers: q_full, q_empty, k_full[KS], v_full[VS], s_full[2],
+  // p_full[2], o_done[2], o_free, mma_done, and the
   // (m, l) exchange barriers of the two softmax groups: lbar[4]
-  static constexpr int NBAR = 2 + 2 * KS + 2 * VS + 8 + 4;
-  static constexpr int OFF_RED = OFF_BAR + NBAR * 8;
-  // red_m[2 item parity][2 groups][128 rows], red_l[same] (fp32)
-  static constexpr int OFF_MISC = OFF_RED + 2 * (2 * 2 * 128) * 4;
+  static constexpr int NBAR = 2 + KS + VS + 8 + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;  // room to align the base to 1024
 };
@@ -324,12 +332,11 @@ __device__ __forceinline__ void mask_half(float (&x)[64], const HalfInfo<UNIT>& 
 
 struct SoftmaxShared {
   uint64_t* s_full;  // [2]: S buffer J holds the logits of the current tile of parity J
-  uint64_t* p_full;  // [2]: 256 arrivals, P of the tile in S buffer J is in TMEM
+  uint64_t* p_full;  // [2]: 8 arrivals (one per softmax warp), P of the tile in
+                     // S buffer J is in TMEM
   uint64_t* o_done;  // [2]: the PV into O_J of the last committed tile has completed
-  uint64_t* o_free;  // 256 arrivals: both O accumulators have been read out
-  uint64_t* lbar;    // [4 quadrants], 64 arrivals: (m, l) exchange of an item
-  float* red_m;      // [2 item parity][2 groups][128 rows]
-  float* red_l;      // [2 item parity][2 groups][128 rows]
+  uint64_t* o_free;  // 8 arrivals: both O accumulators have been read out
+  uint64_t* lbar;    // [4 quadrants], 2 arrivals: (m, l) exchange of an item
   volatile int* abort;
 };
 
@@ -337,43 +344,72 @@ __device__ __forceinline__ float nan_flag() { return __int_as_float(0x7fc00000);
 
 // Exponentials of one 64-column half: p = 2^(x*scale_log2 + off[s]) with the
 // offset off[s] = log-weight - m of the column's slot (W columns each), packed
-// to bf16 pairs; returns the sum of the rounded values.  The scale-and-shift
-// and the running sums use the paired fp32 instructions (two lanes of work
-// per instruction).
+// to bf16 pairs; the row sum adds the rounded values.  The scale-and-shift and
+// the running sums use the paired fp32 instructions (two lanes of work per
+// instruction).  The packed pairs are stored into TMEM at taddr (this
+// thread's lane) in two 16-word chunks as they are formed, so that the first
+// chunk's store overlaps the second chunk's arithmetic.  Also returns, in
+// amax, the largest exponent argument: the tile's maximum relative to the
+// maximum the offsets were formed with (-inf when every column is masked).
 template <int W>
-__device__ __forceinline__ float exp_pack_half(const float (&x)[64], float scale_log2,
-                                               const float (&off)[64 / W], bool simple,
-                                               uint32_t (&pk)[32]) {
+__device__ __forceinline__ float exp_store_half(const float (&x)[64], float scale_log2,
+                                                const float (&off)[64 / W], bool simple,
+                                                uint32_t taddr, float& amax) {
   const float2 sl = make_float2(scale_log2, scale_log2);
   float2 acc[4];
+  float mx[4];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) acc[j] = make_float2(0.f, 0.f);
+  for (int j = 0; j < 4; ++j) {
+    acc[j] = make_float2(0.f, 0.f);
+    mx[j] = -INFINITY;
+  }
 #pragma unroll
-  for (int c = 0; c < 64; c += 2) {
-    const float o = off[c / W];
-    const float2 arg = __ffma2_rn(make_float2(x[c], x[c + 1]), sl, make_float2(o, o));
-    float p0, p1;
+  for (int ch = 0; ch < 2; ++ch) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = ch * 32 + 2 * i;
+      const float o = off[c / W];
+      const float2 arg = __ffma2_rn(make_float2(x[c], x[c + 1]), sl, make_float2(o, o));
+      mx[i & 3] = fmax3(mx[i & 3], arg.x, arg.y);
+      float p0, p1;
 #if STA_POLY_EVERY > 0
-    // one pair in every STA_POLY_EVERY on the FMA pipe (finite arguments only)
-    if (simple && ((c >> 1) % STA_POLY_EVERY) == STA_POLY_EVERY - 1) {
-      p0 = exp2_poly(arg.x);
-      p1 = exp2_poly(arg.y);
-    } else {
+      if (simple && (i % STA_POLY_EVERY) == STA_POLY_EVERY - 1) {
+        p0 = exp2_poly(arg.x);
+        p1 = exp2_poly(arg.y);
+      } else {
+        p0 = fast_exp2(arg.x);
+        p1 = fast_exp2(arg.y);
+      }
+#else
+      (void)simple;
       p0 = fast_exp2(arg.x);
       p1 = fast_exp2(arg.y);
-    }
-#else
-    (void)simple;
-    p0 = fast_exp2(arg.x);
-    p1 = fast_exp2(arg.y);
 #endif
-    pk[c >> 1] = pack_bf16x2(p0, p1);
-    acc[(c >> 1) & 3] =
-        __fadd2_rn(acc[(c >> 1) & 3], make_float2(bf16_lo(pk[c >> 1]), bf16_hi(pk[c >> 1])));
+      pk[i] = pack_bf16x2(p0, p1);
+      acc[i & 3] = __fadd2_rn(acc[i & 3], make_float2(bf16_lo(pk[i]), bf16_hi(pk[i])));
+    }
+    tmem_st16(taddr + ch * 16, pk);
   }
+  amax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
   const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
   const float2 t = __fadd2_rn(s01, s23);
   return t.x + t.y;
+}
+
+// O_J *= f (this thread's row): D/32 chunks of 32 columns through registers.
+template <int D>
+__device__ __forceinline__ void rescale_o(uint32_t tO, float f) {
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t v[32];
+    tmem_ld32(tO + ch * 32, v);
+    tmem_wait_ld();
+    tmem_regs_ready(v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+    tmem_st32(tO + ch * 32, v);
+  }
 }
 
 // Largest logit of each W-column slot.
@@ -429,7 +465,7 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
   uint32_t g = 0, nitem = 0;
   bool ok = true;
   for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
-    if (*abort) break;
+    if (__any_sync(0xffffffffu, *abort != 0)) break;
     const Item I = decode_item(a, it);
     int tok = -1;
     if (I.kind == kItemGatherDense) {
@@ -489,7 +525,8 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         load_half_raw<UNIT>(a, I, t + 1, J, raw_next);  // next tile's entries
       }
       const bool simple = full && !weighted && !window;  // no mask, no weight
-      if (!mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit)) {
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit))) {
         ok = false;
         break;
       }
@@ -516,68 +553,111 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         bias[q] = (weighted && static_cast<unsigned>(raw.u[q]) < static_cast<unsigned>(n_units))
                       ? raw.lw[q] * inv_scale
                       : 0.f;
-      float ms[NS];
-      slot_max<SW>(x, ms);
-      float mraw = ms[0] + bias[0];
+#if STA_SPEC_MAX
+      // Speculative maximum: once every row of the warp has a finite running
+      // maximum, the exponentials are formed against it straight away and
+      // the tile's maximum comes out of the same pass; a row whose maximum
+      // rose by more than the deferral threshold (the condition under which
+      // O_J is rescaled) forms them again after the rescale.
+      const bool spec = __all_sync(0xffffffffu, m_run != -INFINITY);
+#else
+      const bool spec = false;
+#endif
+      if (!spec) {
+        float ms[NS];
+        slot_max<SW>(x, ms);
+        float mraw = ms[0] + bias[0];
 #pragma unroll
-      for (int q = 1; q < NS; ++q) mraw = fmaxf(mraw, ms[q] + bias[q]);
-      const float m_tile = mraw * scale_log2;  // -inf if all masked
-      const float m_new = fmaxf(m_run, m_tile);
-      const bool need = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
-      if (__any_sync(0xffffffffu, need)) {
-        // O_J holds tiles < t of this item; the last of them (tile gg - 1)
-        // must be accumulated before O_J is rescaled.
-        const uint32_t gp = gg - 1;
-        if (!mbar_wait(sh.o_done + (gp & 1), (gp >> 1) & 1, abort, limit)) {
-          ok = false;
-          break;
+        for (int q = 1; q < NS; ++q) mraw = fmaxf(mraw, ms[q] + bias[q]);
+        const float m_tile = mraw * scale_log2;  // -inf if all masked
+        const float m_new = fmaxf(m_run, m_tile);
+        const bool need = (m_run != -INFINITY) && (m_new > m_run + kRescaleThreshold);
+        if (__any_sync(0xffffffffu, need)) {
+          // O_J holds tiles < t of this item; the last of them (tile gg - 1)
+          // must be accumulated before O_J is rescaled.
+          const uint32_t gp = gg - 1;
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(sh.o_done + (gp & 1), (gp >> 1) & 1, abort, limit))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          rescale_o<D>(tO, need ? fast_exp2(m_run - m_new) : 1.f);
+          tmem_wait_st();
+          if (need) {
+            l_run *= fast_exp2(m_run - m_new);
+            m_run = m_new;
+          }
         }
-        tc_fence_after();
-        const float f = need ? fast_exp2(m_run - m_new) : 1.f;
-#pragma unroll
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t v[32];
-          tmem_ld32(tO + ch * 32, v);
-          tmem_wait_ld();
-          tmem_regs_ready(v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
-          tmem_st32(tO + ch * 32, v);
-        }
-        tmem_wait_st();
-        if (need) {
-          l_run *= f;
-          m_run = m_new;
-        }
+        if (m_run == -INFINITY) m_run = m_new;
       }
-      if (m_run == -INFINITY) m_run = m_new;
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
       // P of this group's 64 keys, packed over the first 32 of its (already
       // read) logit columns
-      uint32_t pk[32];
       float off[NS];
 #pragma unroll
       for (int q = 0; q < NS; ++q) off[q] = fmaf(bias[q], scale_log2, -m_use);
-      l_run += exp_pack_half<SW>(x, scale_log2, off, simple, pk);
-      tmem_st32(tS + J * 64, pk);
+      float amax;
+      float lsum = exp_store_half<SW>(x, scale_log2, off, simple, tS + J * 64, amax);
+      if (spec) {
+        const bool redo = amax > kRescaleThreshold;
+        if (__any_sync(0xffffffffu, redo)) {
+          const uint32_t gp = gg - 1;  // as above: t >= 1 here
+          if (!__all_sync(0xffffffffu,
+                          mbar_wait(sh.o_done + (gp & 1), (gp >> 1) & 1, abort, limit))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = redo ? fast_exp2(-amax) : 1.f;
+          rescale_o<D>(tO, f);
+          tmem_wait_st();  // also orders the first pass's P stores before the second's
+          if (redo) {
+            l_run *= f;
+            m_run += amax;
+#pragma unroll
+            for (int q = 0; q < NS; ++q) off[q] -= amax;
+          }
+          lsum = exp_store_half<SW>(x, scale_log2, off, simple, tS + J * 64, amax);
+        }
+      }
+      l_run += lsum;
+      // One arrival per warp, after every lane's stores have completed (a
+      // barrier word takes its arrivals one at a time).
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(sh.p_full + sb);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sh.p_full + sb);
     }
     if (!ok) break;
     // ------------------------------------------------------------ epilogue
     const uint32_t gl = g + I.ntiles - 1;  // last tile of the item
-    // (m, l) slots alternate with the item parity: the partner may still be
-    // reading the previous item's slot when this group gets here.
-    const int slot = (nitem & 1) * 256;
-    sh.red_m[slot + J * 128 + r] = m_run;
-    sh.red_l[slot + J * 128 + r] = l_run;
-    mbar_arrive(sh.lbar + quad);
-    bool okw = mbar_wait(sh.lbar + quad, nitem & 1, abort, limit);
-    const float mo = sh.red_m[slot + (1 - J) * 128 + r];
-    const float lo = sh.red_l[slot + (1 - J) * 128 + r];
+    // The two groups exchange (m, l) of each row through TMEM: group J
+    // writes its pair into columns 64J+32, 64J+33 of the last tile's S
+    // buffer (its own half, which only it reads and has already read; the
+    // tile's P, which its PV still reads, is in columns 64J..64J+31), at the
+    // row's lane.  The MMA issuer writes the buffer again (the QK of tile
+    // gl+2) only after both groups have finished this epilogue (o_free).
+    const uint32_t tX = tmem + lane_off + (gl & 1) * 128 + 32;
+    tmem_st2(tX + 64 * J, __float_as_uint(m_run), __float_as_uint(l_run));
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sh.lbar + quad);
+    bool okw = __all_sync(0xffffffffu, mbar_wait(sh.lbar + quad, nitem & 1, abort, limit));
+    float mo = 0.f, lo = 0.f;
+    if (okw) {
+      tc_fence_after();
+      uint32_t um, ul;
+      tmem_ld2(tX + 64 * (1 - J), um, ul);
+      tmem_wait_ld();
+      mo = __uint_as_float(um);
+      lo = __uint_as_float(ul);
+    }
     // the commit after the item's last PV covers every earlier MMA
-    if (okw) okw = mbar_wait(sh.o_done + (gl & 1), (gl >> 1) & 1, abort, limit);
+    if (okw)
+      okw = __all_sync(0xffffffffu,
+                       mbar_wait(sh.o_done + (gl & 1), (gl >> 1) & 1, abort, limit));
     g += I.ntiles;
     ++nitem;
     if (!okw) {
@@ -629,7 +709,8 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       }
     }
     tc_fence_before();
-    mbar_arrive(sh.o_free);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sh.o_free);
   }
   if (!ok) fail(abort, a.dev_status);
 }
@@ -665,6 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_k_il,
                     const __grid_constant__ CUtensorMap tm_v_il) {
   using L = Layout<D, KS, VS>;
+  static_assert(KS == 2 && VS == 2, "ring slots are released by the S-full / O-done commits");
   // d = 128 with 16-key units: list tiles use the interleaved layout
   // [8-row group][half][8 rows][128 B], one TMA copy per unit (two 2 KB
   // copies per unit, one per half, measured 18% slower; from 32 keys up the
@@ -681,17 +763,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars + 0;
   uint64_t* q_empty = bars + 1;
   uint64_t* k_full = bars + 2;
-  uint64_t* k_empty = k_full + KS;
-  uint64_t* v_full = k_empty + KS;
-  uint64_t* v_empty = v_full + VS;
-  uint64_t* s_full = v_empty + VS;
+  uint64_t* v_full = k_full + KS;
+  uint64_t* s_full = v_full + VS;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* o_free = o_done + 2;
   uint64_t* mma_done = o_free + 1;
   uint64_t* lbar = mma_done + 1;  // [4]
-  float* red_m = reinterpret_cast<float*>(smem + L::OFF_RED);
-  float* red_l = red_m + 2 * 2 * 128;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -703,20 +781,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(q_empty, 1);
     for (int i = 0; i < KS; ++i) {
       mbar_init(k_full + i, 1);
-      mbar_init(k_empty + i, 1);
     }
     for (int i = 0; i < VS; ++i) {
       mbar_init(v_full + i, 1);
-      mbar_init(v_empty + i, 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(s_full + i, 1);
-      mbar_init(p_full + i, 256);  // both softmax groups write P of every tile
+      mbar_init(p_full + i, 8);  // both softmax groups write P of every tile
       mbar_init(o_done + i, 1);
     }
-    mbar_init(o_free, 256);
+    mbar_init(o_free, 8);
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 4; ++i) mbar_init(lbar + i, 64);
+    for (int i = 0; i < 4; ++i) mbar_init(lbar + i, 2);
     *abort = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tm_q);
@@ -741,53 +817,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   int dummy_abort_storage = 0;
   volatile int* no_abort = &dummy_abort_storage;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // K/V tiles are read by every query block of a head: keep them in L2
-    // ahead of the Q tiles, which are read once.
+  if (warp == 0 || warp == kWarpV) {
+    // ----------------------------------------------------------- producers
+    // Warp 0 loads the Q tile of each item and the K tiles, warp kWarpV the
+    // V tiles, each into its own ring, so that a V copy never waits behind
+    // a K slot.  K/V tiles are read by every query block of a head: keep
+    // them in L2 ahead of the Q tiles, which are read once.
+    const bool is_v = (warp == kWarpV);
     const uint64_t pol_kv = l2_policy_evict_last();
     const uint64_t pol_q = l2_policy_evict_first();
-    uint32_t kt = 0, vt = 0, qn = 0;
+    const uint32_t RS = is_v ? VS : KS;
+    uint64_t* ring_full = is_v ? v_full : k_full;
+    // Slot n % 2 of the K ring is free once the QK of tile n-2 has
+    // completed, which is the S-full commit of that tile (S buffer n % 2);
+    // likewise the V ring's slot once the PV of tile n-2 has completed (its
+    // O-done commit).  The next phase of either barrier needs tile n's copy,
+    // so a wait can never see a phase further on.  Sharing the commits
+    // halves the tcgen05.commit count per tile.
+    uint64_t* ring_empty = is_v ? o_done : s_full;
+    uint8_t* ring = is_v ? sV : sK;
+    const CUtensorMap* m_il = is_v ? &tm_v_il : &tm_k_il;
+    uint32_t n = 0, qn = 0;  // tiles issued into the ring, items
+    int ok = 1;
     for (int it = blockIdx.x; it < a.n_items; it += gridDim.x) {
-      if (*abort) break;
+      if (__any_sync(0xffffffffu, *abort != 0)) break;
       const Item I = decode_item(a, it);
       if (I.ntiles == 0) continue;
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(q_empty, (qn & 1) ^ 1, abort, limit);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) {
-        if (lane == 0) fail(abort, a.dev_status);
-        break;
-      }
-      if (I.kind == kItemGatherDense) {
-        // Gather the routed query rows and store them in the 128-byte
-        // swizzled layout TMA would produce (16-byte chunk c of row r sits
-        // at chunk c ^ (r % 8) of the row).
-        const __nv_bfloat16* qh = a.q + static_cast<size_t>(I.head) * a.N * D;
-        for (int r = lane; r < kTileQ; r += 32) {
-          const int src_r = (r < I.q_len) ? r : 0;
-          const int tok = __ldg(a.routed_ids + I.gbase + src_r);
-          const uint4* src = reinterpret_cast<const uint4*>(qh + static_cast<size_t>(tok) * D);
-#pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
-            const int h = c >> 3, cc = c & 7;
-            uint4 val = __ldg(src + c);
-            *reinterpret_cast<uint4*>(sQ + h * kHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = val;
-          }
+      if (!is_v) {
+        if (lane == 0) ok = mbar_wait(q_empty, (qn & 1) ^ 1, abort, limit);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) fail(abort, a.dev_status);
+          break;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(q_full);
-      } else if (lane == 0) {
-        mbar_arrive_expect_tx(q_full, L::TILE_BYTES);
+        if (I.kind == kItemGatherDense) {
+          // Gather the routed query rows and store them in the 128-byte
+          // swizzled layout TMA would produce (16-byte chunk c of row r sits
+          // at chunk c ^ (r % 8) of the row).
+          const __nv_bfloat16* qh = a.q + static_cast<size_t>(I.head) * a.N * D;
+          for (int r = lane; r < kTileQ; r += 32) {
+            const int src_r = (r < I.q_len) ? r : 0;
+            const int tok = __ldg(a.routed_ids + I.gbase + src_r);
+            const uint4* src = reinterpret_cast<const uint4*>(qh + static_cast<size_t>(tok) * D);
 #pragma unroll
-        for (int h = 0; h < L::DH; ++h)
-          tma_load_3d_hint(sQ + h * kHalfBytes, &tm_q, q_full, h * 64, I.q_start, I.head, pol_q);
+            for (int c = 0; c < D / 8; ++c) {
+              const int h = c >> 3, cc = c & 7;
+              uint4 val = __ldg(src + c);
+              *reinterpret_cast<uint4*>(sQ + h * kHalfBytes + r * 128 + ((cc ^ (r & 7)) << 4)) =
+                  val;
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(q_full);
+        } else if (lane == 0) {
+          mbar_arrive_expect_tx(q_full, L::TILE_BYTES);
+#pragma unroll
+          for (int h = 0; h < L::DH; ++h)
+            tma_load_3d_hint(sQ + h * kHalfBytes, &tm_q, q_full, h * 64, I.q_start, I.head,
+                             pol_q);
+        }
+        ++qn;
       }
-      ++qn;
       const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
-      const CUtensorMap* mk = dense_like ? &tm_k_f : &tm_k_u;
-      const CUtensorMap* mv = dense_like ? &tm_v_f : &tm_v_u;
+      const CUtensorMap* mt =
+          dense_like ? (is_v ? &tm_v_f : &tm_k_f) : (is_v ? &tm_v_u : &tm_k_u);
       const int unit = I.unit;
       const bool il = kInterleaved && !dense_like;
       const int nops = il ? I.upt : I.upt * L::DH;
@@ -801,44 +895,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           float lw;
           bool bad;
           u = slot_unit(a, I, t, s, nv, lw, bad);
-          if (bad) raise_status(a.dev_status, STA_DEV_BAD_INDEX);
+          if (bad && !is_v) raise_status(a.dev_status, STA_DEV_BAD_INDEX);
         }
-        // K
-        {
-          const int st = kt % KS;
-          if (lane == 0) ok = mbar_wait(k_empty + st, ((kt / KS) & 1) ^ 1, abort, limit);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
-          if (lane == 0) mbar_arrive_expect_tx(k_full + st, L::TILE_BYTES);
-          __syncwarp();
-          if (il) {
-            if (lane < nops)
-              load_unit_il<UNIT>(sK + st * L::TILE_BYTES, &tm_k_il, mk, k_full + st, s, u, n_il,
-                           I.head, pol_kv);
-          } else if (lane < nops) {
-            tma_load_3d_hint(sK + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mk,
-                             k_full + st, h * 64, u * unit, I.head, pol_kv);
-          }
-          ++kt;
+        const uint32_t st = n % RS;
+        if (lane == 0) ok = mbar_wait(ring_empty + st, ((n / RS) & 1) ^ 1, abort, limit);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) mbar_arrive_expect_tx(ring_full + st, L::TILE_BYTES);
+        __syncwarp();
+        if (il) {
+          if (lane < nops)
+            load_unit_il<UNIT>(ring + st * L::TILE_BYTES, m_il, mt, ring_full + st, s, u, n_il,
+                               I.head, pol_kv);
+        } else if (lane < nops) {
+          tma_load_3d_hint(ring + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mt,
+                           ring_full + st, h * 64, u * unit, I.head, pol_kv);
         }
-        // V
-        {
-          const int st = vt % VS;
-          if (lane == 0) ok = mbar_wait(v_empty + st, ((vt / VS) & 1) ^ 1, abort, limit);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
-          if (!ok) break;
-          if (lane == 0) mbar_arrive_expect_tx(v_full + st, L::TILE_BYTES);
-          __syncwarp();
-          if (il) {
-            if (lane < nops)
-              load_unit_il<UNIT>(sV + st * L::TILE_BYTES, &tm_v_il, mv, v_full + st, s, u, n_il,
-                           I.head, pol_kv);
-          } else if (lane < nops) {
-            tma_load_3d_hint(sV + st * L::TILE_BYTES + h * kHalfBytes + s * unit * 128, mv,
-                             v_full + st, h * 64, u * unit, I.head, pol_kv);
-          }
-          ++vt;
-        }
+        ++n;
       }
       if (!ok) {
         if (lane == 0) fail(abort, a.dev_status);
@@ -846,12 +919,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     // Let every copy this warp issued land before the CTA can exit.
-    if (lane == 0) {
-      for (uint32_t i = (kt > KS ? kt - KS : 0); i < kt; ++i)
-        mbar_wait(k_full + (i % KS), (i / KS) & 1, no_abort, limit);
-      for (uint32_t i = (vt > VS ? vt - VS : 0); i < vt; ++i)
-        mbar_wait(v_full + (i % VS), (i / VS) & 1, no_abort, limit);
-    }
+    if (lane == 0)
+      for (uint32_t i = (n > RS ? n - RS : 0); i < n; ++i)
+        mbar_wait(ring_full + (i % RS), (i / RS) & 1, no_abort, limit);
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
@@ -861,21 +931,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
       uint32_t kt = 0, vt = 0, qn = 0, g = 0;
       bool ok = true;
-      // first: the next PV starts the accumulators O_0 / O_1 of this item;
-      // wait_free: O_0/O_1 still hold the previous item until both softmax
-      // groups have read them out (o_free).
+      // first: the next PV starts the accumulators O_0 / O_1 of this item.
+      // O_0/O_1 and the (m, l) exchange columns of an item's last S buffer
+      // stay in use until both softmax groups have finished the item's
+      // epilogue (o_free, one phase per item): nfree counts the phases seen.
+      // The first PV of item qn, and the QK into the last S buffer of item
+      // qn-1 (tile xtile = its last tile + 2), wait for epilogues 0..qn-1.
       bool first = true;
-      bool wait_free = false;
+      uint32_t nfree = 0, xtile = 0xffffffffu;
+      auto ensure_free = [&](uint32_t k) -> bool {
+        while (nfree < k) {
+          if (!mbar_wait(o_free, nfree & 1, abort, limit)) return false;
+          ++nfree;
+        }
+        return true;
+      };
       // K/V tiles of the current item are in the interleaved layout: 8-row
       // groups 2048 bytes apart, halves 1024 apart (else 1024 and 16384)
       bool il = false;
       auto issue_pv = [&](uint32_t gg) -> bool {
         const uint32_t sb = gg & 1;
         if (!mbar_wait(p_full + sb, (gg >> 1) & 1, abort, limit)) return false;
-        if (wait_free) {
-          if (!mbar_wait(o_free, (qn - 1) & 1, abort, limit)) return false;
-          wait_free = false;
-        }
+        if (first && !ensure_free(qn)) return false;
         tc_fence_after();
         const int st = vt % VS;
         if (!mbar_wait(v_full + st, (vt / VS) & 1, abort, limit)) return false;
@@ -895,7 +972,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ts(tO, pa, bdesc, IDESC_PV, (first && (kk & 3) == 0) ? 0u : 1u);
         }
         first = false;
-        mma_commit(v_empty + st);
         ++vt;
         mma_commit(o_done + sb);
         return true;
@@ -910,11 +986,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         first = true;
-        wait_free = qn > 0;
         il = kInterleaved && (I.kind == kItemList || I.kind == kItemLocal);
         for (int t = 0; t < I.ntiles; ++t) {
           const int st = kt % KS;
           if (!mbar_wait(k_full + st, (kt / KS) & 1, abort, limit)) {
+            ok = false;
+            break;
+          }
+          if (g + t == xtile && !ensure_free(qn)) {
             ok = false;
             break;
           }
@@ -931,7 +1010,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                    : smem_desc_sw128(kbase + off, 16, 1024);
             mma_bf16_ss(tS, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
           }
-          mma_commit(k_empty + st);
           ++kt;
           mma_commit(s_full + sb);
           if (t == I.ntiles - 1) mma_commit(q_empty);
@@ -947,6 +1025,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++qn;
         g += I.ntiles;
+        xtile = g + 1;
       }
       if (!ok) fail(abort, a.dev_status);
       // all issued MMAs complete before TMEM is released
@@ -954,9 +1033,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0, no_abort, limit);
     }
     __syncwarp();
-  } else {
+  } else if (warp < kWarpV) {
     // ------------------------------------------------------------- softmax
-    SoftmaxShared sh{s_full, p_full, o_done, o_free, lbar, red_m, red_l, abort};
+    SoftmaxShared sh{s_full, p_full, o_done, o_free, lbar, abort};
     // one copy of the softmax code serves both groups (J is a runtime value)
     softmax_role<D, UNIT>(a, sh, tmem, warp, lane, warp < 6 ? 0 : 1);
   }
