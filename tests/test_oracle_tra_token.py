@@ -1,0 +1,140 @@
+"""Pins of the token-level entropy -> radius -> block selector oracle
+("Token Radius Attention for Efficient Video Generation", 2. Methodology:
+Insight I, Insight II, The TRA Pipeline), against closed forms, invariants
+and brute force on tiny grids."""
+import math
+
+import numpy as np
+
+from oracle import tra_token
+
+
+def test_entropy_of_equal_logits_is_ln_n():
+    rng = np.random.default_rng(0)
+    q = rng.normal(size=(5, 8))
+    k = np.tile(rng.normal(size=(1, 8)), (37, 1))  # every key identical
+    H = tra_token.query_entropy(q, k, 0.3)
+    assert np.allclose(H, math.log(37), atol=1e-12)
+
+
+def test_entropy_of_one_dominant_logit_is_near_zero():
+    q = np.zeros((1, 4))
+    q[0, 0] = 1.0
+    k = np.zeros((50, 4))
+    k[7, 0] = 200.0  # logit 200 against 0 for the 49 others
+    H = tra_token.query_entropy(q, k, 1.0)
+    # exact value: p = 1/(1 + 49 e^-200); H ~ 49 * 200 * e^-200
+    assert 0.0 <= H[0] < 1e-80
+
+
+def test_entropy_equals_loops():
+    rng = np.random.default_rng(1)
+    q = rng.normal(size=(3, 6))
+    k = rng.normal(size=(11, 6))
+    s = 0.7
+    H = tra_token.query_entropy(q, k, s)
+    for i in range(3):
+        logits = [s * sum(q[i, t] * k[j, t] for t in range(6)) for j in range(11)]
+        mx = max(logits)
+        w = [math.exp(x - mx) for x in logits]
+        z = sum(w)
+        ref = -sum((x / z) * math.log(x / z) for x in w)
+        assert abs(H[i] - ref) < 1e-12
+
+
+def test_radius_without_decay_is_uniform():
+    F, tau, H = 7, 3.0, 2.5
+    r2 = tra_token.radius2(H, 2, F, tau, 0.0)
+    r0sq = tau * math.exp(H) / (math.pi * F)
+    assert np.allclose(r2, r0sq, rtol=1e-14)
+    # the disks of all frames hold n = tau e^H tokens in the continuous sense
+    assert abs(math.pi * r2.sum() - tau * math.exp(H)) < 1e-9
+
+
+def test_radius_decay_by_frame_distance():
+    F, gamma = 9, 0.4
+    r2 = tra_token.radius2(1.0, 4, F, 2.0, gamma)
+    for f in range(F):
+        assert abs(r2[f] / r2[4] - math.exp(-2 * gamma * abs(f - 4))) < 1e-14
+    G = sum(math.exp(-2 * gamma * abs(f - 4)) for f in range(F))
+    assert abs(math.pi * r2.sum() - 2.0 * math.e) < 1e-9 * G
+
+
+def _gauss_circle(r2):
+    """Lattice points (x, y) with x^2 + y^2 <= r2."""
+    R = int(math.isqrt(int(math.floor(r2))))
+    return sum(2 * int(math.isqrt(int(math.floor(r2 - x * x)))) + 1 for x in range(-R, R + 1))
+
+
+def test_kept_count_is_the_gauss_circle_count():
+    F, Hh, W = 1, 41, 41
+    i = 20 * W + 20  # centre of the frame: no edge clipping
+    for H in (0.5, 2.0, 3.7):
+        kept, _ = tra_token.key_keep(i, H, F, Hh, W, 1.0, 0.0)
+        r2 = math.exp(H) / math.pi
+        assert kept.sum() == _gauss_circle(r2)
+
+
+def _brute_lists(H, F, Hh, W, B, tau, gamma, vote):
+    N = F * Hh * W
+    nb = (N + B - 1) // B
+    S = Hh * W
+    out = {}
+    for qb in range(nb):
+        cnt = [0] * nb
+        for i in range(qb * B, min(N, qb * B + B)):
+            fi, hi, wi = i // S, (i % S) // W, i % W
+            G = sum(math.exp(-2 * gamma * abs(f - fi)) for f in range(F))
+            r0sq = tau * math.exp(H[i]) / (math.pi * G)
+            for j in range(N):
+                fj, hj, wj = j // S, (j % S) // W, j % W
+                rf = r0sq * math.exp(-2 * gamma * abs(fj - fi))
+                if (hj - hi) ** 2 + (wj - wi) ** 2 <= rf:
+                    cnt[j // B] += 1
+        out[qb] = [kb for kb in range(nb) if cnt[kb] >= vote]
+    return out
+
+
+def test_block_lists_equal_brute_force():
+    rng = np.random.default_rng(3)
+    F, Hh, W, B = 3, 5, 7, 16  # N = 105: partial last block
+    H = rng.uniform(0.0, 3.0, size=F * Hh * W)
+    for vote in (1, 3):
+        got = tra_token.block_lists(H, F, Hh, W, B, 1.5, 0.35, vote)
+        ref = _brute_lists(H, F, Hh, W, B, 1.5, 0.35, vote)
+        for qb in ref:
+            ids, amb = got[qb]
+            assert set(ids.tolist()) ^ set(ref[qb]) <= set(amb.tolist())
+            assert list(ids) == sorted(ids)
+
+
+def test_huge_budget_keeps_everything():
+    F, Hh, W, B = 2, 4, 6, 8
+    H = np.zeros(F * Hh * W)
+    got = tra_token.block_lists(H, F, Hh, W, B, 1e6, 0.0, 1)
+    nb = (F * Hh * W + B - 1) // B
+    assert all(list(ids) == list(range(nb)) for ids, _ in got.values())
+
+
+def test_tiny_budget_keeps_the_query_column():
+    # r^2 < 1 in every frame: only the key at the query's own (h, w) of each
+    # frame is kept
+    F, Hh, W, B = 3, 4, 4, 4
+    N = F * Hh * W
+    H = np.zeros(N)
+    got = tra_token.block_lists(H, F, Hh, W, B, 1e-3, 0.2, 1)
+    S = Hh * W
+    for qb, (ids, amb) in got.items():
+        want = set()
+        for i in range(qb * B, min(N, qb * B + B)):
+            s = i % S
+            for f in range(F):
+                want.add((f * S + s) // B)
+        assert set(ids.tolist()) == want and len(amb) == 0
+
+
+def test_vote_above_pair_count_is_empty():
+    F, Hh, W, B = 2, 3, 3, 6
+    H = np.ones(F * Hh * W)
+    got = tra_token.block_lists(H, F, Hh, W, B, 1.0, 0.1, vote=10 ** 6)
+    assert all(len(ids) == 0 for ids, _ in got.values())
