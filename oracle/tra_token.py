@@ -18,26 +18,31 @@ Readings (the page prints no formulas beyond the two above):
 1. H_i is the natural-log entropy of the dense softmax of query i over all N
    keys with scale 1/sqrt(d).
 2. n_i = tau * exp(H_i).
-3. The base radius r0 makes the disks of all frames hold n_i tokens in the
-   continuous approximation: sum_f pi (r0 phi(|f - f_i|))^2 = n_i, so
-   r0^2 = n_i / (pi * G(f_i)) with G(f_i) = sum_{f=0}^{F-1} exp(-2 gamma |f - f_i|).
-   Frame f's squared radius is r_f^2 = r0^2 * exp(-2 gamma |f - f_i|).
-4. Key j in frame f_j is kept for query i iff (h_j - h_i)^2 + (w_j - w_i)^2
-   <= r_{f_j}^2 (latent grid units).  d^2 = 0 always passes, so every frame
-   keeps at least the key at the query's own (h, w).
+3. The budget is shared among the frames as disks whose radius decays by
+   phi: frame f gets n_f = n_i * exp(-2 gamma |f - f_i|) / G(f_i) tokens,
+   G(f_i) = sum_{f=0}^{F-1} exp(-2 gamma |f - f_i|), as a disk of squared
+   radius r_f^2 = n_f / pi = r0^2 * exp(-2 gamma |f - f_i|) with
+   r0^2 = n_i / (pi * G(f_i)) (so sum_f pi r_f^2 = n_i).
+4. A frame whose share is below one token (n_f < 1) keeps no key;
+   otherwise key j in frame f_j is kept for query i iff
+   (h_j - h_i)^2 + (w_j - w_i)^2 <= r_{f_j}^2 (latent grid units).  (Without
+   the share rule every frame would keep the key at the query's own (h, w),
+   however small its disk: a tube through all frames that alone keeps ~16%
+   of the block pairs at the Wan shape, whatever the entropies.)
 5. Token voting: key block kb is kept for query block qb iff at least `vote`
    kept (i, j) pairs have i in qb and j in kb.
-Near-threshold pairs: |d^2 - r_f^2| <= NEAR * r_f^2 (relative: r_f^2 carries
-the rounding of exp(H)).  A block whose decision depends on such pairs is
-reported separately (block_lists returns the ambiguous blocks).
+Near-threshold pairs: |d^2 - r_f^2| <= NEAR * r_f^2 or |n_f - 1| <= NEAR
+(relative: r_f^2 and n_f carry the rounding of exp(H)).  A block whose
+decision depends on such pairs is reported separately (block_lists returns
+the ambiguous blocks).
 
 Parity: pinned (tests/test_oracle_tra_token.py): entropy is ln N for equal
 logits and ~0 for one dominant logit and equals a pure-Python loop; gamma = 0
 gives r0^2 = n / (pi F) and equal per-frame radii; the kept-key count of a
 query far from the frame edges equals the Gauss circle count; block lists
 equal a brute-force loop over all token pairs on tiny grids; a huge tau keeps
-every block and a tiny tau keeps only the blocks holding the query's own
-(h, w) column; vote thresholds above the pair count give empty lists.
+every block, a tiny tau keeps nothing, and a steep decay keeps only the
+query's own frame; vote thresholds above the pair count give empty lists.
 """
 import numpy as np
 
@@ -82,8 +87,9 @@ def key_keep(i, H_i, F, Hh, W, tau, gamma):
     fj, hj, wj = coords(np.arange(N), F, Hh, W)
     d2 = (hj - hi).astype(np.float64) ** 2 + (wj - wi).astype(np.float64) ** 2
     rf = r2[fj]
-    kept = d2 <= rf
-    near = np.abs(d2 - rf) <= NEAR * rf
+    share = np.pi * rf  # n_f: the frame's share of the budget
+    kept = (share >= 1.0) & (d2 <= rf)
+    near = (np.abs(d2 - rf) <= NEAR * rf) | (np.abs(share - 1.0) <= NEAR)
     return kept, near
 
 

@@ -89,7 +89,7 @@ def _brute_lists(H, F, Hh, W, B, tau, gamma, vote):
             for j in range(N):
                 fj, hj, wj = j // S, (j % S) // W, j % W
                 rf = r0sq * math.exp(-2 * gamma * abs(fj - fi))
-                if (hj - hi) ** 2 + (wj - wi) ** 2 <= rf:
+                if math.pi * rf >= 1.0 and (hj - hi) ** 2 + (wj - wi) ** 2 <= rf:
                     cnt[j // B] += 1
         out[qb] = [kb for kb in range(nb) if cnt[kb] >= vote]
     return out
@@ -116,21 +116,24 @@ def test_huge_budget_keeps_everything():
     assert all(list(ids) == list(range(nb)) for ids, _ in got.values())
 
 
-def test_tiny_budget_keeps_the_query_column():
-    # r^2 < 1 in every frame: only the key at the query's own (h, w) of each
-    # frame is kept
+def test_tiny_budget_keeps_nothing():
+    # every frame's share of the budget is below one token
     F, Hh, W, B = 3, 4, 4, 4
-    N = F * Hh * W
-    H = np.zeros(N)
+    H = np.zeros(F * Hh * W)
     got = tra_token.block_lists(H, F, Hh, W, B, 1e-3, 0.2, 1)
+    assert all(len(ids) == 0 and len(amb) == 0 for ids, amb in got.values())
+
+
+def test_steep_decay_keeps_only_the_query_frame():
+    # gamma = 5: the neighbouring frames' shares are e^-10 of the own frame's
+    F, Hh, W, B = 3, 6, 6, 6
+    N = F * Hh * W
     S = Hh * W
+    H = np.full(N, math.log(20.0))  # n = 20 keys, ~all in the own frame
+    got = tra_token.block_lists(H, F, Hh, W, B, 1.0, 5.0, 1)
     for qb, (ids, amb) in got.items():
-        want = set()
-        for i in range(qb * B, min(N, qb * B + B)):
-            s = i % S
-            for f in range(F):
-                want.add((f * S + s) // B)
-        assert set(ids.tolist()) == want and len(amb) == 0
+        frames = {int(kb) * B // S for kb in ids}
+        assert frames == {qb * B // S} and len(amb) == 0
 
 
 def test_vote_above_pair_count_is_empty():
