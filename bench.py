@@ -40,7 +40,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "effective TFLOP/s on retained blocks; speedup vs dense at same shape (1×B200)"
 DEFAULT_WORKLOAD = "wan_radial"
-WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled")
+WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled", "tra_token")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 * 1024 * 1024
 
@@ -219,7 +219,7 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
     fraction.  Returns effective TFLOP/s over the sampled retained pairs."""
     import numpy as np
 
-    from oracle import entropy, ibcs_sip, radial, routed
+    from oracle import entropy, ibcs_sip, radial, routed, tra_token
     from oracle.grid import n_blocks
     from oracle.pipeline import block_sparse_rows, routed_rows
     from synthetic import make_difficulty, make_qkv
@@ -257,12 +257,31 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
         c = w["ibcs"]
         kbar, n_j = ibcs_sip.subblock_means(kh, U)
         t_sel_per_item = (time.perf_counter() - t0) / nqb  # one head's sub-block means
+    elif sel == "tra_token":
+        c = w["tra_token"]
+        Hq = np.zeros(N)
+        t_lists = 0.0
     budget_end = time.perf_counter() + budget_s
     t_att = 0.0
     for qb in order:
         qb = int(qb)
         ts = time.perf_counter()
-        if sel == "ibcs_sip":
+        if sel == "tra_token":
+            # the entropies are the warm-up's (not charged to the step); the
+            # block lists and the attention are
+            lo, hi = qb * B, min(N, qb * B + B)
+            Hq[lo:hi] = tra_token.query_entropy(qh[lo:hi], kh, 1.0 / np.sqrt(d))
+            ts = time.perf_counter()
+            ids, _ = tra_token.block_lists(Hq, w["F"], w["H"], w["W"], B, c["tau"], c["gamma"],
+                                           c["vote"], [qb])[qb]
+            t_lists += time.perf_counter() - ts
+            ts = time.perf_counter()
+            block_sparse_rows(qh, kh, vh, qb, ids, B, U)
+            t_att += time.perf_counter() - ts
+            keys = sum(min(U, N - u * U) for u in ids)
+            flops += 4.0 * d * (hi - lo) * keys
+            t_sel_per_item = t_lists / (done + 1)
+        elif sel == "ibcs_sip":
             lo, hi = qb * B, min(N, qb * B + B)
             row = ibcs_sip.select_row(qh[lo:hi], kbar, n_j, c["seed"], qb, c["k"], c["iters"],
                                       c["sample_frac"])
@@ -336,7 +355,7 @@ def config_of(w):
 
 
 # ------------------------------------------------------------------- GPU arm
-SELECTOR_LAUNCHES = {"radial": 1, "entropy": 2, "routed": 2, "ibcs_sip": 5}
+SELECTOR_LAUNCHES = {"radial": 1, "entropy": 2, "routed": 2, "ibcs_sip": 5, "tra_token": 1}
 
 
 def selector_bytes(w, lists_entries):
@@ -350,6 +369,8 @@ def selector_bytes(w, lists_entries):
         return 2 * h * N * d * 2 + 8 * lists_entries, "fma (fp32 importance GEMM)"
     if sel == "routed":
         return 4 * N + 5 * N + 4 * lists_entries, "latency"
+    if sel == "tra_token":
+        return 4 * h * N + 4 * lists_entries, "alu (disk counting per query and key block)"
     return 4 * lists_entries, "launch"
 
 
@@ -372,7 +393,27 @@ def main(argv=None):
     difd = dif.cuda() if routed else None
     od = torch.empty_like(qd)
     prob = session.problem(w)
-    sel = session.selector(w, difd)
+    # token-level TRA: the per-query entropies come from a dense warm-up pass
+    # (dense attention that also writes each query's entropy), run once and
+    # reused by every step, as the pipeline reuses them across denoising steps
+    ent = None
+    warm = None
+    if w["selector"] == "tra_token":
+        ent = torch.empty(w["heads"], w["N"], dtype=torch.float32, device="cuda")
+        ow = torch.empty_like(qd)
+        stw = torch.zeros(1, dtype=torch.int32, device="cuda")
+        for i in range(4):
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record()
+            sta.sta_dense_attn_entropy_fwd(session.problem(w), qd, kd, vd, 0.0, ow, ent,
+                                           dev_status=stw)
+            b_.record()
+            torch.cuda.synchronize()
+            warm = a_.elapsed_time(b_)
+        if int(stw.item()) != 0:
+            raise RuntimeError("device status " + sta.sta_dev_status_string(int(stw.item())))
+        del ow
+    sel = session.selector(w, difd, entropy=ent)
     prm = session.attn_params(w)
     L = session.Lists(w)
     sws = session.selector_workspace(w)
@@ -508,6 +549,11 @@ def main(argv=None):
         "gpu_launches": (SELECTOR_LAUNCHES[w["selector"]] + 1) * args.steps,
         "clocks": clk.summary(),
     }
+    if warm is not None:
+        dflops = 4.0 * w["d"] * float(w["N"]) ** 2 * w["heads"]
+        line["tra_warmup"] = {"ms": warm, "tflops": dflops / (warm * 1e-3) / 1e12,
+                              "note": "dense attention + per-query entropy, run once and "
+                                      "reused by the steps (not in the timed step)"}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget_s)
     if rank == 0:

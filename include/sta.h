@@ -74,7 +74,8 @@ typedef enum {
   STA_SEL_RADIAL = 0,    /* static radial window         [RAD] The idea behind Radial Attention */
   STA_SEL_ENTROPY = 1,   /* pooled entropy -> radius     [TRA] 2. Methodology, The TRA Pipeline */
   STA_SEL_IBCS_SIP = 2,  /* k-means importance + Philox inclusion-probability sampling  [AB]   */
-  STA_SEL_ROUTED = 3     /* difficulty routing: dense for the top fraction, local window [HETA] */
+  STA_SEL_ROUTED = 3,    /* difficulty routing: dense for the top fraction, local window [HETA] */
+  STA_SEL_TRA_TOKEN = 4  /* per-query entropy -> budget -> disk radius -> token voting  [TRA]  */
 } sta_selector;
 
 /* Problem geometry.  N = F*H*W tokens per head. */
@@ -105,6 +106,17 @@ typedef struct {
  *          ties to the lower index) attend to all keys; every other token
  *          attends to keys with |df| <= win_f, dh in [-win_h, win_h),
  *          dw in [-win_w, win_w).  `difficulty` is a device pointer [N].
+ * tra_token [TRA] 2. Methodology (Insight I, Insight II, The TRA Pipeline):
+ *          tra_entropy is a device pointer [heads][N] of per-query attention
+ *          entropies in nats (from sta_dense_attn_entropy_fwd, the dense
+ *          warm-up).  Query i keeps about n_i = tau * exp(H_i) keys, laid out
+ *          as a disk per frame: r0^2 = n_i / (pi * sum_f exp(-2 gamma |f - f_i|)),
+ *          r_f^2 = r0^2 * exp(-2 gamma |f - f_i|) (fp32); frame f holds
+ *          pi * r_f^2 tokens of the budget and keeps nothing when that is
+ *          below 1; otherwise key j is kept iff
+ *          (h_j - h_i)^2 + (w_j - w_i)^2 <= r_{f_j}^2.  A key block is listed
+ *          for a query block iff at least tra_vote kept (query, key) pairs fall
+ *          in the pair (token voting).  block_q == kv_unit; lists per head.
  */
 typedef struct {
   sta_selector kind;
@@ -123,6 +135,10 @@ typedef struct {
   float dense_frac;
   int win_f, win_h, win_w;
   const float* difficulty;
+  /* tra_token */
+  float tra_tau, tra_gamma;
+  int tra_vote;
+  const float* tra_entropy;
 } sta_selector_params;
 
 /*
@@ -220,6 +236,20 @@ sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void
                               const void* v, float scale, void* o,
                               void* workspace, size_t workspace_bytes,
                               int32_t* dev_status, sta_stream_t stream);
+
+/*
+ * Dense attention that also writes each query's attention entropy
+ * ([TRA] 2. Methodology, The TRA Pipeline: entropy is taken during a dense
+ * warm-up pass and feeds the STA_SEL_TRA_TOKEN selector):
+ *   entropy[h][i] = -sum_j p_ij ln p_ij,  p_ij = softmax_j(scale * q_i.k_j)
+ * in nats, accumulated in fp32 from the unrounded probabilities.  entropy:
+ * device float [heads][N], caller-owned.  Other arguments, results and
+ * errors as sta_dense_attn_fwd.
+ */
+sta_status sta_dense_attn_entropy_fwd(const sta_problem* prob, const void* q, const void* k,
+                                      const void* v, float scale, void* o, float* entropy,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, sta_stream_t stream);
 
 /*
  * sta_sparse_attn_fwd with no workspace argument, for callers that cannot

@@ -22,7 +22,7 @@ STA_DEV_BAD_INDEX = 0x8
 STA_DEV_RANGE = 0x10
 
 STA_BF16, STA_F32 = 0, 1
-STA_SEL_RADIAL, STA_SEL_ENTROPY, STA_SEL_IBCS_SIP, STA_SEL_ROUTED = 0, 1, 2, 3
+STA_SEL_RADIAL, STA_SEL_ENTROPY, STA_SEL_IBCS_SIP, STA_SEL_ROUTED, STA_SEL_TRA_TOKEN = 0, 1, 2, 3, 4
 STA_ATTN_LISTS, STA_ATTN_ROUTED = 0, 1
 
 
@@ -42,7 +42,9 @@ class SelectorParams(ctypes.Structure):
                 ("sample_frac", ctypes.c_float), ("seed", ctypes.c_uint64),
                 ("dense_frac", ctypes.c_float), ("win_f", ctypes.c_int),
                 ("win_h", ctypes.c_int), ("win_w", ctypes.c_int),
-                ("difficulty", ctypes.c_void_p)]
+                ("difficulty", ctypes.c_void_p),
+                ("tra_tau", ctypes.c_float), ("tra_gamma", ctypes.c_float),
+                ("tra_vote", ctypes.c_int), ("tra_entropy", ctypes.c_void_p)]
 
 
 class BlockLists(ctypes.Structure):
@@ -84,6 +86,12 @@ SIGNATURES = {
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                           ctypes.c_void_p, ctypes.c_void_p]),
+    "sta_dense_attn_entropy_fwd": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_void_p,
+                                                  ctypes.c_void_p, ctypes.c_void_p,
+                                                  ctypes.c_float, ctypes.c_void_p,
+                                                  ctypes.c_void_p, ctypes.c_void_p,
+                                                  ctypes.c_size_t, ctypes.c_void_p,
+                                                  ctypes.c_void_p]),
     "sta_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sta_dev_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "sta_version": (ctypes.c_int, []),

@@ -88,6 +88,20 @@ def sta_dense_attn_fwd(prob, q, k, v, scale, o, workspace=None, workspace_bytes=
                                  _ptr(dev_status), _stream(stream)), "sta_dense_attn_fwd")
 
 
+def sta_dense_attn_entropy_fwd(prob, q, k, v, scale, o, entropy, workspace=None,
+                               workspace_bytes=0, dev_status=None, stream=None):
+    """Dense attention plus each query's attention entropy (nats) into
+    `entropy` [heads, N] float32: the dense warm-up of the token-level
+    selector."""
+    lib = _lib.load()
+    if isinstance(workspace, torch.Tensor) and not workspace_bytes:
+        workspace_bytes = workspace.numel() * workspace.element_size()
+    check(lib.sta_dense_attn_entropy_fwd(ctypes.byref(prob), _ptr(q), _ptr(k), _ptr(v),
+                                         float(scale), _ptr(o), _ptr(entropy), _ptr(workspace),
+                                         workspace_bytes, _ptr(dev_status), _stream(stream)),
+          "sta_dense_attn_entropy_fwd")
+
+
 def sta_status_string(code: int) -> str:
     return _lib.load().sta_status_string(code).decode()
 

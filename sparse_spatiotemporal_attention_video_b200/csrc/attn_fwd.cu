@@ -351,13 +351,15 @@ __device__ __forceinline__ float nan_flag() { return __int_as_float(0x7fc00000);
 // chunk's store overlaps the second chunk's arithmetic.  Also returns, in
 // amax, the largest exponent argument: the tile's maximum relative to the
 // maximum the offsets were formed with (-inf when every column is masked).
-template <int W>
+template <int W, bool ENT = false>
 __device__ __forceinline__ float exp_store_half(const float (&x)[64], float scale_log2,
                                                 const float (&off)[64 / W], bool simple,
-                                                uint32_t taddr, float& amax) {
+                                                uint32_t taddr, float& amax, float& zt,
+                                                float& at) {
   const float2 sl = make_float2(scale_log2, scale_log2);
   float2 acc[4];
   float mx[4];
+  float2 ez = make_float2(0.f, 0.f), ea = make_float2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     acc[j] = make_float2(0.f, 0.f);
@@ -388,9 +390,18 @@ __device__ __forceinline__ float exp_store_half(const float (&x)[64], float scal
 #endif
       pk[i] = pack_bf16x2(p0, p1);
       acc[i & 3] = __fadd2_rn(acc[i & 3], make_float2(bf16_lo(pk[i]), bf16_hi(pk[i])));
+      if constexpr (ENT) {
+        // entropy terms from the unrounded p: sum p and sum p * (y - m) (log2
+        // units; masked columns have p = 0 and a clamped argument)
+        const float2 pp = make_float2(p0, p1);
+        ez = __fadd2_rn(ez, pp);
+        ea = __ffma2_rn(pp, make_float2(fmaxf(arg.x, -256.f), fmaxf(arg.y, -256.f)), ea);
+      }
     }
     tmem_st16(taddr + ch * 16, pk);
   }
+  zt = ez.x + ez.y;
+  at = ea.x + ea.y;
   amax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
   const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
   const float2 t = __fadd2_rn(s01, s23);
@@ -449,7 +460,7 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
 // Softmax warpgroup J (4 warps): keys [64J, 64J+64) of every tile, query
 // row r = 32*quadrant + lane per thread, accumulator O_J (see the file
 // comment).
-template <int D, int UNIT>
+template <int D, int UNIT, bool ENT>
 __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxShared& sh,
                                              uint32_t tmem, int warp, int lane, int J) {
   constexpr int OH = D / 2;     // output columns per group
@@ -504,6 +515,7 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
     const int n_full = a.N / UNIT;  // units whose keys all lie below N
     const int n_units = (a.N + UNIT - 1) / UNIT;
     float m_run = -INFINITY, l_run = 0.f;
+    float z_run = 0.f, a_run = 0.f;  // entropy terms (ENT): sum p, sum p (y - m)
     HalfRaw<UNIT> raw_next;
     if (!dense_like) load_half_raw<UNIT>(a, I, 0, J, raw_next);
     for (int t = 0; t < I.ntiles; ++t) {
@@ -585,7 +597,12 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
           rescale_o<D>(tO, need ? fast_exp2(m_run - m_new) : 1.f);
           tmem_wait_st();
           if (need) {
-            l_run *= fast_exp2(m_run - m_new);
+            const float f = fast_exp2(m_run - m_new);
+            l_run *= f;
+            if constexpr (ENT) {
+              a_run = f * fmaf(m_run - m_new, z_run, a_run);
+              z_run *= f;
+            }
             m_run = m_new;
           }
         }
@@ -597,8 +614,8 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       float off[NS];
 #pragma unroll
       for (int q = 0; q < NS; ++q) off[q] = fmaf(bias[q], scale_log2, -m_use);
-      float amax;
-      float lsum = exp_store_half<SW>(x, scale_log2, off, simple, tS + J * 64, amax);
+      float amax, zt, at;
+      float lsum = exp_store_half<SW, ENT>(x, scale_log2, off, simple, tS + J * 64, amax, zt, at);
       if (spec) {
         const bool redo = amax > kRescaleThreshold;
         if (__any_sync(0xffffffffu, redo)) {
@@ -614,14 +631,22 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
           tmem_wait_st();  // also orders the first pass's P stores before the second's
           if (redo) {
             l_run *= f;
+            if constexpr (ENT) {
+              a_run = f * fmaf(-amax, z_run, a_run);
+              z_run *= f;
+            }
             m_run += amax;
 #pragma unroll
             for (int q = 0; q < NS; ++q) off[q] -= amax;
           }
-          lsum = exp_store_half<SW>(x, scale_log2, off, simple, tS + J * 64, amax);
+          lsum = exp_store_half<SW, ENT>(x, scale_log2, off, simple, tS + J * 64, amax, zt, at);
         }
       }
       l_run += lsum;
+      if constexpr (ENT) {
+        z_run += zt;
+        a_run += at;
+      }
       // One arrival per warp, after every lane's stores have completed (a
       // barrier word takes its arrivals one at a time).
       tmem_wait_st();
@@ -640,19 +665,23 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
     // gl+2) only after both groups have finished this epilogue (o_free).
     const uint32_t tX = tmem + lane_off + (gl & 1) * 128 + 32;
     tmem_st2(tX + 64 * J, __float_as_uint(m_run), __float_as_uint(l_run));
+    if constexpr (ENT) tmem_st2(tX + 64 * J + 2, __float_as_uint(z_run), __float_as_uint(a_run));
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sh.lbar + quad);
     bool okw = __all_sync(0xffffffffu, mbar_wait(sh.lbar + quad, nitem & 1, abort, limit));
-    float mo = 0.f, lo = 0.f;
+    float mo = 0.f, lo = 0.f, zo = 0.f, ao = 0.f;
     if (okw) {
       tc_fence_after();
-      uint32_t um, ul;
+      uint32_t um, ul, uz = 0, ua = 0;
       tmem_ld2(tX + 64 * (1 - J), um, ul);
+      if constexpr (ENT) tmem_ld2(tX + 64 * (1 - J) + 2, uz, ua);
       tmem_wait_ld();
       mo = __uint_as_float(um);
       lo = __uint_as_float(ul);
+      zo = __uint_as_float(uz);
+      ao = __uint_as_float(ua);
     }
     // the commit after the item's last PV covers every earlier MMA
     if (okw)
@@ -675,6 +704,25 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
     const float inv_l = empty ? 0.f : 1.f / l_tot;
     const float c0 = f0 * inv_l, c1 = f1 * inv_l;
     if (J == 0 && active && empty) raise_status(a.dev_status, STA_DEV_EMPTY_ROW);
+    if constexpr (ENT) {
+      // H = ln Z - ln 2 * A / Z over both groups' keys, with Z = sum p and
+      // A = sum p (y - m) brought to the common maximum m (log2 units)
+      if (J == 0 && active && a.entropy) {
+        const float z0 = J == 0 ? z_run : zo, z1 = J == 0 ? zo : z_run;
+        const float a0 = J == 0 ? a_run : ao, a1 = J == 0 ? ao : a_run;
+        float Z = 0.f, A = 0.f;
+        if (f0 > 0.f) {
+          Z = fmaf(f0, z0, Z);
+          A = fmaf(f0, fmaf(m0 - m, z0, a0), A);
+        }
+        if (f1 > 0.f) {
+          Z = fmaf(f1, z1, Z);
+          A = fmaf(f1, fmaf(m1 - m, z1, a1), A);
+        }
+        const float H = Z > 0.f ? logf(Z) - 0.6931471805599453f * (A / Z) : 0.f;
+        a.entropy[orow] = H;
+      }
+    }
 #pragma unroll
     for (int ch = 0; ch < OH / 32; ++ch) {
       const uint32_t col = tmem + lane_off + 256 + OB + ch * 32;
@@ -736,7 +784,7 @@ __device__ __forceinline__ void load_unit_il(uint8_t* tile, const CUtensorMap* m
   }
 }
 
-template <int D, int KS, int VS, int UNIT>
+template <int D, int KS, int VS, int UNIT, bool ENT>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k_u,
@@ -1037,7 +1085,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- softmax
     SoftmaxShared sh{s_full, p_full, o_done, o_free, lbar, abort};
     // one copy of the softmax code serves both groups (J is a runtime value)
-    softmax_role<D, UNIT>(a, sh, tmem, warp, lane, warp < 6 ? 0 : 1);
+    softmax_role<D, UNIT, ENT>(a, sh, tmem, warp, lane, warp < 6 ? 0 : 1);
   }
 
   tc_fence_before();
@@ -1055,14 +1103,14 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
   }
 }
 
-template <int D, int KS, int VS, int UNIT>
+template <int D, int KS, int VS, int UNIT, bool ENT = false>
 cudaError_t launch_t(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tku,
                      const CUtensorMap& tvu, const CUtensorMap& tkf, const CUtensorMap& tvf,
                      const CUtensorMap& tki, const CUtensorMap& tvi, int num_sms,
                      cudaStream_t stream) {
   using L = Layout<D, KS, VS>;
-  auto kern = attn_fwd_kernel<D, KS, VS, UNIT>;
-  cudaError_t e = set_dyn_smem<attn_fwd_kernel<D, KS, VS, UNIT>>(L::ALLOC);
+  auto kern = attn_fwd_kernel<D, KS, VS, UNIT, ENT>;
+  cudaError_t e = set_dyn_smem<attn_fwd_kernel<D, KS, VS, UNIT, ENT>>(L::ALLOC);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
@@ -1077,6 +1125,17 @@ cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tq,
                              const CUtensorMap& tkf, const CUtensorMap& tvf,
                              const CUtensorMap& tki, const CUtensorMap& tvi, int num_sms,
                              cudaStream_t stream) {
+  // dense attention with per-query entropy (the dense warm-up)
+  if (a.entropy) {
+    if (a.mode != kModeDense || a.unit != kTileK) return cudaErrorInvalidValue;
+    if (d == 128)
+      return launch_t<128, STA_KSTAGES, STA_VSTAGES, 128, true>(a, tq, tku, tvu, tkf, tvf, tki,
+                                                                tvi, num_sms, stream);
+    if (d == 64)
+      return launch_t<64, STA_KSTAGES, STA_VSTAGES, 128, true>(a, tq, tku, tvu, tkf, tvf, tki,
+                                                               tvi, num_sms, stream);
+    return cudaErrorInvalidValue;
+  }
 #define STA_ATTN_CASE(DD, UU)                                                              \
   if (d == DD && a.unit == UU)                                                             \
     return launch_t<DD, STA_KSTAGES, STA_VSTAGES, UU>(a, tq, tku, tvu, tkf, tvf, tki, tvi, \

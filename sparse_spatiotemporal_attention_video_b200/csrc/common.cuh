@@ -58,6 +58,7 @@ struct AttnArgs {
   void* o;
   int out_f32;
   int32_t* dev_status;
+  float* entropy;  // dense mode: per-query attention entropy [heads][N] (nats), or null
 };
 
 // Launchers (attn_fwd.cu).  With d = 128 and 16-key units the
@@ -109,6 +110,14 @@ cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, float* sc
                                  int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
                                  float* entropy, int32_t* radius, int32_t* dev_status,
                                  cudaStream_t s);
+
+// Token-level entropy -> disk radius -> token voting (sel_tra.cu).
+int tra_max_frames();
+int tra_max_block();
+cudaError_t launch_tra_token_lists(const float* entropy, int heads, int F, int H, int W, int B,
+                                   float tau, float gamma, int vote, int32_t* idx, int32_t* cnt,
+                                   int cap, int32_t* required_cap, int32_t* dev_status,
+                                   cudaStream_t s);
 
 // Difficulty routing (sel_routed.cu).
 cudaError_t launch_routed_select(const float* difficulty, int N, int n_routed,

@@ -1,0 +1,192 @@
+// sel_tra.cu -- token-level entropy -> budget -> disk radius -> token voting.
+//
+// "Token Radius Attention for Efficient Video Generation", 2. Methodology:
+// Insight I (the token budget follows the query's attention entropy,
+// B ~ tau * exp(H) / N, so query i keeps about n_i = tau * exp(H_i) keys),
+// Insight II (the kept keys form a query-centred spatial disk whose radius
+// shrinks with temporal distance by exp(-gamma * delta)) and The TRA Pipeline
+// (entropy from a dense warm-up -> budget -> base radius -> per-frame 2D disk
+// -> token voting into block-sparse lists):
+//
+//   r0^2  = tau * exp(H_i) / (pi * G(f_i)),  G(f) = sum_f' exp(-2 gamma |f' - f|)
+//   r_f^2 = r0^2 * exp(-2 gamma |f - f_i|)                          (fp32)
+//   frame f's share of the budget is n_f = pi * r_f^2 tokens; a frame with
+//   n_f < 1 keeps no key, otherwise
+//   key j kept for query i  iff  (h_j - h_i)^2 + (w_j - w_i)^2 <= r_{f_j}^2
+//   key block kb listed for query block qb iff at least `vote` kept pairs
+//   (i in qb, j in kb).
+//
+// One CTA per (query block, head).  The block's queries (coordinates and
+// r0^2) and the per-distance decay table are staged in shared memory; thread
+// t then takes key blocks t, t + 256, ...: it splits the block's tokens into
+// grid-row segments [w0, w1] of one (f, h) and, per query, counts the keys
+// of each segment inside the query's disk: with rest = r_f^2 - dh^2 >= 0
+// (exact in fp32: dh^2 is an integer below 2^24) and dw = floor(sqrt(rest))
+// (corrected so that dw^2 <= rest < (dw+1)^2 exactly), the row's kept
+// columns are [w_i - dw, w_i + dw].  A segment is skipped without visiting
+// the queries when no query can reach it: per frame, the largest r_f^2 over
+// the block's queries (frames whose share is below one token excluded)
+// against the squared row distance from the block's row span.  Kept blocks
+// are compacted in ascending order with warp ballots and a block-wide scan.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+
+namespace sta {
+namespace {
+
+constexpr int kTraThreads = 256;
+constexpr int kTraMaxQ = 128;   // query block size limit
+constexpr int kTraMaxF = 1024;  // frame count limit (decay table)
+
+struct TraArgs {
+  const float* entropy;  // [heads][N]
+  int heads, F, H, W, B, nb;
+  float tau, gamma;
+  int vote;
+  int32_t* idx;
+  int32_t* cnt;
+  int cap;
+  int32_t* required_cap;
+  int32_t* dev_status;
+};
+
+// Largest integer dw >= 0 with dw^2 <= t, for 0 <= t < W^2 (the squares
+// are compared in double, exactly).
+__device__ __forceinline__ int floor_sqrt(float t) {
+  long long dw = static_cast<long long>(sqrtf(t));
+  while (static_cast<double>((dw + 1) * (dw + 1)) <= static_cast<double>(t)) ++dw;
+  while (dw > 0 && static_cast<double>(dw * dw) > static_cast<double>(t)) --dw;
+  return static_cast<int>(dw);
+}
+
+__global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraArgs a) {
+  __shared__ float decay[kTraMaxF];    // exp(-2 gamma delta), delta = |f - f_i|
+  __shared__ float qr0[kTraMaxQ];      // r0^2 of each query of the block
+  __shared__ int qf[kTraMaxQ], qh[kTraMaxQ], qw[kTraMaxQ];
+  __shared__ float reach[kTraMaxF];   // per frame: max r_f^2 over the block's queries
+  __shared__ int warp_tot[kTraThreads / 32];
+  __shared__ int running, hmin, hmax;
+  const int qb = blockIdx.x, head = blockIdx.y;
+  const int S = a.H * a.W;
+  const int N = a.F * S;
+  const int q0 = qb * a.B;
+  const int nq = min(a.B, N - q0);
+  for (int dlt = threadIdx.x; dlt < a.F; dlt += kTraThreads)
+    decay[dlt] = expf(-2.0f * a.gamma * static_cast<float>(dlt));
+  if (threadIdx.x == 0) {
+    running = 0;
+    hmin = a.H;
+    hmax = -1;
+  }
+  __syncthreads();
+  const float* Hh = a.entropy + static_cast<size_t>(head) * N;
+  for (int r = threadIdx.x; r < nq; r += kTraThreads) {
+    const int t = q0 + r;
+    const int f = t / S, rem = t - f * S;
+    qf[r] = f;
+    qh[r] = rem / a.W;
+    qw[r] = rem - qh[r] * a.W;
+    float G = 0.f;  // frames in order: the same sum on every query of frame f
+    for (int f2 = 0; f2 < a.F; ++f2) G += decay[abs(f2 - f)];
+    const float n = a.tau * expf(__ldg(Hh + t));
+    qr0[r] = n / (3.14159265358979f * G);
+    atomicMin(&hmin, qh[r]);
+    atomicMax(&hmax, qh[r]);
+  }
+  __syncthreads();
+  for (int f = threadIdx.x; f < a.F; f += kTraThreads) {
+    float m = -1.f;
+    for (int r = 0; r < nq; ++r) {
+      const float rf = qr0[r] * decay[abs(f - qf[r])];
+      if (rf * 3.14159265358979f >= 1.f) m = fmaxf(m, rf);
+    }
+    reach[f] = m;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(head) * a.nb + qb;
+  int32_t* out = a.idx + row * a.cap;
+  for (int c0 = 0; c0 < a.nb; c0 += kTraThreads) {
+    const int kb = c0 + threadIdx.x;
+    bool keep = false;
+    if (kb < a.nb) {
+      const int t0 = kb * a.B, t1 = min(N, t0 + a.B);  // [t0, t1)
+      const float wsq = static_cast<float>(a.W) * static_cast<float>(a.W);
+      int votes = 0;
+      // grid-row segments [w0, w1] of one (f, h) of the key block
+      for (int t = t0; t < t1 && votes < a.vote;) {
+        const int f = t / S, rem = t - f * S;
+        const int h = rem / a.W, w0 = rem - h * a.W;
+        const int w1 = min(a.W - 1, w0 + (t1 - 1 - t));  // inclusive
+        t += w1 - w0 + 1;
+        const int drow = max(0, max(hmin - h, h - hmax));
+        if (static_cast<float>(drow * drow) > reach[f]) continue;  // no query reaches it
+        for (int r = 0; r < nq && votes < a.vote; ++r) {
+          const float rf = qr0[r] * decay[abs(f - qf[r])];
+          if (rf * 3.14159265358979f < 1.f) continue;  // share below one token
+          const int dh = h - qh[r];
+          const float rest = rf - static_cast<float>(dh * dh);
+          if (rest < 0.f) continue;
+          // rest >= W^2: the disk spans the whole row
+          const int dw = rest >= wsq ? a.W : floor_sqrt(rest);
+          const int lo = max(w0, qw[r] - dw), hi_w = min(w1, qw[r] + dw);
+          if (hi_w >= lo) votes += hi_w - lo + 1;
+        }
+      }
+      keep = votes >= a.vote;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    int before = running;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    const int pos = before + __popc(bal & ((1u << lane) - 1u));
+    if (keep && pos < a.cap) out[pos] = kb;
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int w = 0; w < kTraThreads / 32; ++w) running += warp_tot[w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const int total = running;
+    a.cnt[row] = min(total, a.cap);
+    if (a.required_cap) atomicMax(a.required_cap, total);
+    if (total > a.cap) raise_status(a.dev_status, STA_DEV_CAPACITY);
+  }
+}
+
+}  // namespace
+
+int tra_max_frames() { return kTraMaxF; }
+int tra_max_block() { return kTraMaxQ; }
+
+cudaError_t launch_tra_token_lists(const float* entropy, int heads, int F, int H, int W, int B,
+                                   float tau, float gamma, int vote, int32_t* idx, int32_t* cnt,
+                                   int cap, int32_t* required_cap, int32_t* dev_status,
+                                   cudaStream_t s) {
+  TraArgs a;
+  a.entropy = entropy;
+  a.heads = heads;
+  a.F = F;
+  a.H = H;
+  a.W = W;
+  a.B = B;
+  const long long N = static_cast<long long>(F) * H * W;
+  a.nb = static_cast<int>((N + B - 1) / B);
+  a.tau = tau;
+  a.gamma = gamma;
+  a.vote = vote;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.cap = cap;
+  a.required_cap = required_cap;
+  a.dev_status = dev_status;
+  if (a.nb <= 0 || heads <= 0) return cudaSuccess;
+  tra_token_lists_kernel<<<dim3(static_cast<unsigned>(a.nb), static_cast<unsigned>(heads)),
+                           kTraThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace sta

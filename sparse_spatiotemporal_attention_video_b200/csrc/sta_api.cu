@@ -268,6 +268,7 @@ int sta_build_blocks_rows(const sta_problem* prob, const sta_selector_params* se
       return nqb;
     case STA_SEL_ENTROPY:
     case STA_SEL_IBCS_SIP:
+    case STA_SEL_TRA_TOKEN:
       return nqb * prob->heads;
   }
   return -1;
@@ -331,6 +332,21 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
                                       sel->ent_tile_w, out->idx, out->cnt, out->cap,
                                       out->required_cap, out->entropy, out->radius, dev_status,
                                       s)))
+        return STA_ERR_CUDA;
+      return STA_OK;
+    }
+    case STA_SEL_TRA_TOKEN: {
+      if (!sel->tra_entropy) return STA_ERR_ARG;
+      if (!(sel->tra_tau > 0.f) || !(sel->tra_gamma >= 0.f) || sel->tra_vote < 1)
+        return STA_ERR_ARG;
+      if (sel->kv_unit != sel->block_q || sel->block_q > tra_max_block() ||
+          prob->F > tra_max_frames())
+        return STA_ERR_UNSUPPORTED;
+      out->head_shared = 0;
+      if (failed(launch_tra_token_lists(sel->tra_entropy, prob->heads, prob->F, prob->H, prob->W,
+                                        sel->block_q, sel->tra_tau, sel->tra_gamma,
+                                        sel->tra_vote, out->idx, out->cnt, out->cap,
+                                        out->required_cap, dev_status, s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }
@@ -471,9 +487,13 @@ sta_status sta_sparse_attn_fwd(const sta_problem* prob, const sta_attn_params* p
   return run_attention(prob, a, qb, kb, vb, prm->kv_unit, s);
 }
 
-sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void* k,
-                              const void* v, float scale, void* o, void* workspace,
-                              size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+namespace {
+
+// Dense attention, with the per-query entropy written to `entropy` when it is
+// not null (the dense warm-up of the token-level selector).
+sta_status dense_attn(const sta_problem* prob, const void* q, const void* k, const void* v,
+                      float scale, void* o, float* entropy, void* workspace,
+                      size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
   sta_status st = check_problem(prob);
   if (st != STA_OK) return st;
   if (!q || !k || !v || !o) return STA_ERR_ARG;
@@ -489,15 +509,35 @@ sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void
   a.scale_log2 = sc * 1.4426950408889634f;
   a.mode = kModeDense;
   a.block_q = kTileQ;
+  a.unit = kTileK;
   a.n_qb = (N + kTileQ - 1) / kTileQ;
   a.n_items = prob->heads * a.n_qb;
   a.o = o;
   a.out_f32 = prob->dtype == STA_F32;
   a.dev_status = dev_status;
+  a.entropy = entropy;
   const __nv_bfloat16 *qb, *kb, *vb;
   st = stage_inputs(prob, q, k, v, workspace, workspace_bytes, &qb, &kb, &vb, s);
   if (st != STA_OK) return st;
   return run_attention(prob, a, qb, kb, vb, kTileK, s);
+}
+
+}  // namespace
+
+sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void* k,
+                              const void* v, float scale, void* o, void* workspace,
+                              size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  return dense_attn(prob, q, k, v, scale, o, nullptr, workspace, workspace_bytes, dev_status,
+                    stream);
+}
+
+sta_status sta_dense_attn_entropy_fwd(const sta_problem* prob, const void* q, const void* k,
+                                      const void* v, float scale, void* o, float* entropy,
+                                      void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, sta_stream_t stream) {
+  if (!entropy) return STA_ERR_ARG;
+  return dense_attn(prob, q, k, v, scale, o, entropy, workspace, workspace_bytes, dev_status,
+                    stream);
 }
 
 }  // extern "C"

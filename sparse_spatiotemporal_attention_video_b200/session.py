@@ -8,11 +8,11 @@ import torch
 
 from . import api
 from ._lib import (STA_ATTN_LISTS, STA_ATTN_ROUTED, STA_BF16, STA_F32, STA_SEL_ENTROPY,
-                   STA_SEL_IBCS_SIP, STA_SEL_RADIAL, STA_SEL_ROUTED, AttnParams, BlockLists,
-                   Problem, SelectorParams)
+                   STA_SEL_IBCS_SIP, STA_SEL_RADIAL, STA_SEL_ROUTED, STA_SEL_TRA_TOKEN,
+                   AttnParams, BlockLists, Problem, SelectorParams)
 
 _KINDS = {"radial": STA_SEL_RADIAL, "entropy": STA_SEL_ENTROPY, "ibcs_sip": STA_SEL_IBCS_SIP,
-          "routed": STA_SEL_ROUTED}
+          "routed": STA_SEL_ROUTED, "tra_token": STA_SEL_TRA_TOKEN}
 
 
 def problem(w):
@@ -20,7 +20,7 @@ def problem(w):
                    STA_F32 if w["dtype"] == "f32" else STA_BF16)
 
 
-def selector(w, difficulty=None):
+def selector(w, difficulty=None, entropy=None):
     s = SelectorParams()
     s.kind = _KINDS[w["selector"]]
     s.block_q = w["block_q"]
@@ -41,6 +41,11 @@ def selector(w, difficulty=None):
         s.dense_frac, s.win_f, s.win_h, s.win_w = c["dense_frac"], c["win_f"], c["win_h"], c["win_w"]
         if difficulty is not None:
             s.difficulty = difficulty.data_ptr()
+    elif w["selector"] == "tra_token":
+        c = w["tra_token"]
+        s.tra_tau, s.tra_gamma, s.tra_vote = c["tau"], c["gamma"], c["vote"]
+        if entropy is not None:
+            s.tra_entropy = entropy.data_ptr()
     return s
 
 

@@ -15,7 +15,7 @@ noise_block         (lo, hi): per 128-token block the noise std is drawn
 logit_std           Q and K share one scale factor chosen so that the std of
                     q.k/sqrt(d) over random same-head pairs is this value.
 block_q, kv_unit    query block and key/value unit in tokens.
-selector            "radial" | "entropy" | "ibcs_sip" | "routed" | "dense".
+selector            "radial" | "entropy" | "ibcs_sip" | "routed" | "tra_token".
 """
 import copy
 
@@ -50,6 +50,18 @@ WORKLOADS = {
         selector="entropy",
         entropy=dict(alpha=-208.83056640625, beta=38.206417083740234, r_lo=1, r_hi=2,
                      tile_h=8, tile_w=16),
+        seed=0),
+    # Token-level TRA pipeline at the Wan2.1-1.3B shape: per-query entropy
+    # from a dense warm-up, budget tau*exp(H), a disk per frame whose radius
+    # decays by exp(-gamma*delta) with frame distance, token voting into
+    # 128-token block lists.  tau is fixed once from the oracle so that the
+    # blocks keep about 14% of the key blocks, inside the 9-19% the pages
+    # report (tests/golden/make_tra_token_calibration.py; value stored in
+    # tests/golden/tra_token_calibration.json and copied here).
+    "tra_token": dict(
+        heads=12, F=21, H=30, W=52, d=128, dtype="bf16", noise=0.5,
+        noise_block=None, logit_std=3.0, block_q=128, kv_unit=128,
+        selector="tra_token", tra_token=dict(tau=0.07146470248699188, gamma=0.25, vote=1),
         seed=0),
     # HetA-style routing at the Wan2.2-5B shape 31x44x80 (N=109120), 24 heads.
     # Top 20% of tokens by a Beta(2,5) difficulty go to dense attention; the
