@@ -46,8 +46,8 @@ L2_FLUSH_BYTES = 256 * 1024 * 1024
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for
 # the kernel source it was taken on (sha256 of attn_fwd.cu, first 16 hex).
-NCU_TRAFFIC = {"source_sha": "594603df108c44a5", "workload": "wan_radial",
-               "bytes_per_launch": 304205568 + 84179200}
+NCU_TRAFFIC = {"source_sha": "8c8e5398b9d4d3c5", "workload": "wan_radial",
+               "bytes_per_launch": 302877440 + 84381696}
 
 
 def parse(argv=None):
