@@ -40,7 +40,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "effective TFLOP/s on retained blocks; speedup vs dense at same shape (1×B200)"
 DEFAULT_WORKLOAD = "wan_radial"
-WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled", "tra_token")
+WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled", "tra_token",
+             "dynrad_static", "dynrad_dynamic")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 * 1024 * 1024
 
@@ -219,7 +220,7 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
     fraction.  Returns effective TFLOP/s over the sampled retained pairs."""
     import numpy as np
 
-    from oracle import entropy, ibcs_sip, radial, routed, tra_token
+    from oracle import dynrad, entropy, ibcs_sip, radial, routed, tra_token
     from oracle.grid import n_blocks
     from oracle.pipeline import block_sparse_rows, routed_rows
     from synthetic import make_difficulty, make_qkv
@@ -261,6 +262,13 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
         c = w["tra_token"]
         Hq = np.zeros(N)
         t_lists = 0.0
+    elif sel == "dynrad":
+        c = w["dynrad"]
+        got = dynrad.select(qh, kh, w["F"], w["H"], w["W"], B, w["radial"], c["mode"],
+                            c.get("ratio"), c.get("threshold"))
+        lists = {b: ids for b, (ids, _) in got.items()}
+        t_sel_per_item = (time.perf_counter() - t0) / nqb  # one head's selector
+        logw = None
     budget_end = time.perf_counter() + budget_s
     t_att = 0.0
     for qb in order:
@@ -355,7 +363,8 @@ def config_of(w):
 
 
 # ------------------------------------------------------------------- GPU arm
-SELECTOR_LAUNCHES = {"radial": 1, "entropy": 2, "routed": 2, "ibcs_sip": 5, "tra_token": 1}
+SELECTOR_LAUNCHES = {"radial": 1, "entropy": 2, "routed": 2, "ibcs_sip": 5, "tra_token": 1,
+                     "dynrad": 3}
 
 
 def selector_bytes(w, lists_entries):
@@ -363,7 +372,7 @@ def selector_bytes(w, lists_entries):
     entries written (4 B per id, 4 more per log-weight), and the bound."""
     h, N, d = w["heads"], w["N"], w["d"]
     sel = w["selector"]
-    if sel == "entropy":
+    if sel in ("entropy", "dynrad"):
         return 2 * h * N * d * 2 + 4 * lists_entries, "hbm"
     if sel == "ibcs_sip":
         return 2 * h * N * d * 2 + 8 * lists_entries, "fma (fp32 importance GEMM)"
@@ -417,7 +426,7 @@ def main(argv=None):
     prm = session.attn_params(w)
     L = session.Lists(w)
     sws = session.selector_workspace(w)
-    needs_qk = w["selector"] in ("entropy", "ibcs_sip")
+    needs_qk = w["selector"] in ("entropy", "ibcs_sip", "dynrad")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = torch.cuda.current_stream()  # the stream every library call below uses
     l2_flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
@@ -549,6 +558,12 @@ def main(argv=None):
         "gpu_launches": (SELECTOR_LAUNCHES[w["selector"]] + 1) * args.steps,
         "clocks": clk.summary(),
     }
+    # Lists (and, for tra_token, entropies) reused across steps: a step is the
+    # attention alone, timed by its own CUDA graph above.
+    line["list_reuse"] = {"ms_per_step": attn_avg,
+                          "value": total_flops / (max_over_ranks(attn_avg, ws) * 1e-3) / 1e12,
+                          "unit": "TFLOP/s",
+                          "note": "selector run once, its lists reused by every step"}
     if warm is not None:
         dflops = 4.0 * w["d"] * float(w["N"]) ** 2 * w["heads"]
         line["tra_warmup"] = {"ms": warm, "tflops": dflops / (warm * 1e-3) / 1e12,

@@ -75,7 +75,8 @@ typedef enum {
   STA_SEL_ENTROPY = 1,   /* pooled entropy -> radius     [TRA] 2. Methodology, The TRA Pipeline */
   STA_SEL_IBCS_SIP = 2,  /* k-means importance + Philox inclusion-probability sampling  [AB]   */
   STA_SEL_ROUTED = 3,    /* difficulty routing: dense for the top fraction, local window [HETA] */
-  STA_SEL_TRA_TOKEN = 4  /* per-query entropy -> budget -> disk radius -> token voting  [TRA]  */
+  STA_SEL_TRA_TOKEN = 4, /* per-query entropy -> budget -> disk radius -> token voting  [TRA]  */
+  STA_SEL_DYNRAD = 5     /* static-ratio / dynamic-threshold selection in the radial prior [DYN] */
 } sta_selector;
 
 /* Problem geometry.  N = F*H*W tokens per head. */
@@ -117,6 +118,14 @@ typedef struct {
  *          (h_j - h_i)^2 + (w_j - w_i)^2 <= r_{f_j}^2.  A key block is listed
  *          for a query block iff at least tra_vote kept (query, key) pairs fall
  *          in the pair (token voting).  block_q == kv_unit; lists per head.
+ * dynrad   [DYN] Abstract: the radial lists (radial_* parameters) are the
+ *          candidates; p_c = softmax over the candidates of the pooled
+ *          scores Qbar_b.Kbar_c/sqrt(d) (fp32); candidates ranked by score
+ *          (ties to the lower block id).  dyn_mode 0 (static ratio) keeps the
+ *          ceil(dyn_ratio * n) best (relative slack 1e-6, at least 1);
+ *          dyn_mode 1 (dynamic threshold) keeps the shortest best-first
+ *          prefix whose p mass reaches dyn_threshold.  block_q == kv_unit,
+ *          at most 1024 blocks; lists per head, ascending.
  */
 typedef struct {
   sta_selector kind;
@@ -139,6 +148,9 @@ typedef struct {
   float tra_tau, tra_gamma;
   int tra_vote;
   const float* tra_entropy;
+  /* dynrad (and the radial_* fields for its prior) */
+  int dyn_mode;
+  float dyn_ratio, dyn_threshold;
 } sta_selector_params;
 
 /*

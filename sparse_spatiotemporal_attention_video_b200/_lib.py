@@ -22,7 +22,8 @@ STA_DEV_BAD_INDEX = 0x8
 STA_DEV_RANGE = 0x10
 
 STA_BF16, STA_F32 = 0, 1
-STA_SEL_RADIAL, STA_SEL_ENTROPY, STA_SEL_IBCS_SIP, STA_SEL_ROUTED, STA_SEL_TRA_TOKEN = 0, 1, 2, 3, 4
+(STA_SEL_RADIAL, STA_SEL_ENTROPY, STA_SEL_IBCS_SIP, STA_SEL_ROUTED, STA_SEL_TRA_TOKEN,
+ STA_SEL_DYNRAD) = 0, 1, 2, 3, 4, 5
 STA_ATTN_LISTS, STA_ATTN_ROUTED = 0, 1
 
 
@@ -44,7 +45,9 @@ class SelectorParams(ctypes.Structure):
                 ("win_h", ctypes.c_int), ("win_w", ctypes.c_int),
                 ("difficulty", ctypes.c_void_p),
                 ("tra_tau", ctypes.c_float), ("tra_gamma", ctypes.c_float),
-                ("tra_vote", ctypes.c_int), ("tra_entropy", ctypes.c_void_p)]
+                ("tra_vote", ctypes.c_int), ("tra_entropy", ctypes.c_void_p),
+                ("dyn_mode", ctypes.c_int), ("dyn_ratio", ctypes.c_float),
+                ("dyn_threshold", ctypes.c_float)]
 
 
 class BlockLists(ctypes.Structure):

@@ -119,6 +119,14 @@ cudaError_t launch_tra_token_lists(const float* entropy, int heads, int F, int H
                                    int cap, int32_t* required_cap, int32_t* dev_status,
                                    cudaStream_t s);
 
+// Dual-mode selection in the radial prior (sel_dynrad.cu).
+int dynrad_max_candidates();
+cudaError_t launch_dynrad_lists(const float* qbar, const float* kbar, const int32_t* prior_idx,
+                                const int32_t* prior_cnt, int prior_cap, int heads, int nb, int d,
+                                float scale, int mode, float ratio, float threshold, int32_t* idx,
+                                int32_t* cnt, int cap, int32_t* required_cap,
+                                int32_t* dev_status, cudaStream_t s);
+
 // Difficulty routing (sel_routed.cu).
 cudaError_t launch_routed_select(const float* difficulty, int N, int n_routed,
                                  int32_t* routed_ids, uint8_t* routed_flag, cudaStream_t s);

@@ -170,7 +170,7 @@ sta_status run_attention(const sta_problem* p, AttnArgs& a, const __nv_bfloat16*
 
 // Workspace carve-up of the content selectors (256-byte aligned segments).
 struct SelWorkspace {
-  size_t qbar = 0, kbar = 0, scores = 0, cent = 0, wts = 0, p = 0;
+  size_t qbar = 0, kbar = 0, scores = 0, cent = 0, wts = 0, p = 0, prior_idx = 0, prior_cnt = 0;
   size_t kb_hi = 0, kb_lo = 0, c_hi = 0, c_lo = 0, total = 0;
 };
 
@@ -188,7 +188,12 @@ SelWorkspace sel_workspace(const sta_problem* p, const sta_selector_params* sel)
     off += round_up(bytes, 256);
     return at;
   };
-  if (sel->kind == STA_SEL_ENTROPY) {
+  if (sel->kind == STA_SEL_DYNRAD) {
+    w.qbar = take(h * nqb * d * 4);
+    w.kbar = take(h * nku * d * 4);
+    w.prior_idx = take(nqb * nku * 4);
+    w.prior_cnt = take(nqb * 4);
+  } else if (sel->kind == STA_SEL_ENTROPY) {
     w.qbar = take(h * nqb * d * 4);
     w.kbar = take(h * nku * d * 4);
     w.scores = take(h * nqb * nku * 4);
@@ -269,6 +274,7 @@ int sta_build_blocks_rows(const sta_problem* prob, const sta_selector_params* se
     case STA_SEL_ENTROPY:
     case STA_SEL_IBCS_SIP:
     case STA_SEL_TRA_TOKEN:
+    case STA_SEL_DYNRAD:
       return nqb * prob->heads;
   }
   return -1;
@@ -332,6 +338,43 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
                                       sel->ent_tile_w, out->idx, out->cnt, out->cap,
                                       out->required_cap, out->entropy, out->radius, dev_status,
                                       s)))
+        return STA_ERR_CUDA;
+      return STA_OK;
+    }
+    case STA_SEL_DYNRAD: {
+      if (prob->dtype != STA_BF16 || !q || !k) return q && k ? STA_ERR_UNSUPPORTED : STA_ERR_ARG;
+      if (sel->dyn_mode != 0 && sel->dyn_mode != 1) return STA_ERR_ARG;
+      if (sel->dyn_mode == 0 && !(sel->dyn_ratio > 0.f && sel->dyn_ratio <= 1.f))
+        return STA_ERR_ARG;
+      if (sel->dyn_mode == 1 && !(sel->dyn_threshold > 0.f && sel->dyn_threshold <= 1.f))
+        return STA_ERR_ARG;
+      if (sel->kv_unit != sel->block_q) return STA_ERR_UNSUPPORTED;
+      const int S = prob->H * prob->W;
+      if ((sel->block_q + S - 1) / S + 1 > 8) return STA_ERR_UNSUPPORTED;
+      const int N = prob->F * prob->H * prob->W;
+      const int nb = (N + sel->block_q - 1) / sel->block_q;
+      if (nb > dynrad_max_candidates()) return STA_ERR_UNSUPPORTED;
+      const SelWorkspace w = sel_workspace(prob, sel);
+      if (!workspace || workspace_bytes < w.total ||
+          (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return STA_ERR_WORKSPACE;
+      uint8_t* ws = static_cast<uint8_t*>(workspace);
+      float* qbar = reinterpret_cast<float*>(ws + w.qbar);
+      float* kbar = reinterpret_cast<float*>(ws + w.kbar);
+      int32_t* pidx = reinterpret_cast<int32_t*>(ws + w.prior_idx);
+      int32_t* pcnt = reinterpret_cast<int32_t*>(ws + w.prior_cnt);
+      out->head_shared = 0;
+      const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
+      // 1. block means, 2. the radial prior (shared by the heads), 3. selection
+      if (failed(launch_block_means(static_cast<const __nv_bfloat16*>(q),
+                                    static_cast<const __nv_bfloat16*>(k), qbar, kbar,
+                                    prob->heads, N, prob->d, sel->block_q, s)) ||
+          failed(launch_radial_lists(prob->F, prob->H, prob->W, sel->block_q, sel->radial_w0,
+                                     sel->radial_w_off, sel->radial_full_df, pidx, pcnt, nb,
+                                     nullptr, dev_status, s)) ||
+          failed(launch_dynrad_lists(qbar, kbar, pidx, pcnt, nb, prob->heads, nb, prob->d, scale,
+                                     sel->dyn_mode, sel->dyn_ratio, sel->dyn_threshold, out->idx,
+                                     out->cnt, out->cap, out->required_cap, dev_status, s)))
         return STA_ERR_CUDA;
       return STA_OK;
     }

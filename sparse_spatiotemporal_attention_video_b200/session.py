@@ -8,11 +8,11 @@ import torch
 
 from . import api
 from ._lib import (STA_ATTN_LISTS, STA_ATTN_ROUTED, STA_BF16, STA_F32, STA_SEL_ENTROPY,
-                   STA_SEL_IBCS_SIP, STA_SEL_RADIAL, STA_SEL_ROUTED, STA_SEL_TRA_TOKEN,
-                   AttnParams, BlockLists, Problem, SelectorParams)
+                   STA_SEL_DYNRAD, STA_SEL_IBCS_SIP, STA_SEL_RADIAL, STA_SEL_ROUTED,
+                   STA_SEL_TRA_TOKEN, AttnParams, BlockLists, Problem, SelectorParams)
 
 _KINDS = {"radial": STA_SEL_RADIAL, "entropy": STA_SEL_ENTROPY, "ibcs_sip": STA_SEL_IBCS_SIP,
-          "routed": STA_SEL_ROUTED, "tra_token": STA_SEL_TRA_TOKEN}
+          "routed": STA_SEL_ROUTED, "tra_token": STA_SEL_TRA_TOKEN, "dynrad": STA_SEL_DYNRAD}
 
 
 def problem(w):
@@ -25,9 +25,13 @@ def selector(w, difficulty=None, entropy=None):
     s.kind = _KINDS[w["selector"]]
     s.block_q = w["block_q"]
     s.kv_unit = w["kv_unit"]
-    if w["selector"] == "radial":
+    if w["selector"] in ("radial", "dynrad"):
         r = w["radial"]
         s.radial_w0, s.radial_w_off, s.radial_full_df = r["w0"], r["w_off"], r["full_df"]
+    if w["selector"] == "dynrad":
+        c = w["dynrad"]
+        s.dyn_mode = 0 if c["mode"] == "static" else 1
+        s.dyn_ratio, s.dyn_threshold = c.get("ratio", 0.0), c.get("threshold", 0.0)
     elif w["selector"] == "entropy":
         e = w["entropy"]
         s.ent_alpha, s.ent_beta = e["alpha"], e["beta"]

@@ -15,7 +15,8 @@ noise_block         (lo, hi): per 128-token block the noise std is drawn
 logit_std           Q and K share one scale factor chosen so that the std of
                     q.k/sqrt(d) over random same-head pairs is this value.
 block_q, kv_unit    query block and key/value unit in tokens.
-selector            "radial" | "entropy" | "ibcs_sip" | "routed" | "tra_token".
+selector            "radial" | "entropy" | "ibcs_sip" | "routed" | "tra_token" |
+                    "dynrad".
 """
 import copy
 
@@ -62,6 +63,22 @@ WORKLOADS = {
         heads=12, F=21, H=30, W=52, d=128, dtype="bf16", noise=0.5,
         noise_block=None, logit_std=3.0, block_q=128, kv_unit=128,
         selector="tra_token", tra_token=dict(tau=0.07146470248699188, gamma=0.25, vote=1),
+        seed=0),
+    # DynamicRad-style selection inside the radial prior at the Wan2.1-1.3B
+    # shape (the wan_radial lists are the candidates): static ratio keeps the
+    # best 35% of each row's candidates by pooled attention probability,
+    # dynamic threshold the shortest best-first prefix holding 35% of the
+    # mass; both leave about 80% of all block pairs out (the page reports
+    # over 80% effective sparsity).
+    "dynrad_static": dict(
+        heads=12, F=21, H=30, W=52, d=128, dtype="bf16", noise=0.5,
+        noise_block=None, logit_std=3.0, block_q=128, kv_unit=128, selector="dynrad",
+        radial=dict(w0=1560, w_off=1, full_df=-1), dynrad=dict(mode="static", ratio=0.35),
+        seed=0),
+    "dynrad_dynamic": dict(
+        heads=12, F=21, H=30, W=52, d=128, dtype="bf16", noise=0.5,
+        noise_block=None, logit_std=3.0, block_q=128, kv_unit=128, selector="dynrad",
+        radial=dict(w0=1560, w_off=1, full_df=-1), dynrad=dict(mode="dynamic", threshold=0.35),
         seed=0),
     # HetA-style routing at the Wan2.2-5B shape 31x44x80 (N=109120), 24 heads.
     # Top 20% of tokens by a Beta(2,5) difficulty go to dense attention; the
