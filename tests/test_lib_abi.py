@@ -76,3 +76,65 @@ def test_selftest_argument_checks(lib):
     assert lib.sta_selftest_bounded_wait(0, 1, 1, None) == STA_ERR_ARG
     assert lib.sta_selftest_bounded_wait(10**10, 1, 1, None) == STA_ERR_ARG
     assert lib.sta_selftest_bounded_wait(1000, None, 1, None) == STA_ERR_ARG
+
+
+def test_next_selector_argument_checks(lib):
+    """Host checks of the token-level and radial-prior selectors and of the
+    entropy-writing dense entry point; every case returns before a launch."""
+    from sparse_spatiotemporal_attention_video_b200._lib import (
+        STA_ERR_ARG, STA_ERR_UNSUPPORTED, STA_ERR_WORKSPACE, STA_SEL_DYNRAD,
+        STA_SEL_TRA_TOKEN, BlockLists, Problem, SelectorParams)
+    good = Problem(2, 4, 8, 8, 64, 0)  # 2 heads, 256 tokens, two 128-blocks
+    lists = BlockLists()
+    lists.idx, lists.cnt, lists.cap = 256, 512, 4  # never dereferenced on these paths
+    fake = ctypes.c_void_p(4096)
+
+    def build(sel, prob=good, q=fake, k=fake):
+        return lib.sta_build_blocks(ctypes.byref(prob), ctypes.byref(sel), q, k,
+                                    ctypes.byref(lists), None, 0, None, None)
+
+    tra = SelectorParams()
+    tra.kind, tra.block_q, tra.kv_unit = STA_SEL_TRA_TOKEN, 128, 128
+    tra.tra_tau, tra.tra_gamma, tra.tra_vote = 0.07, 0.25, 1
+    assert build(tra) == STA_ERR_ARG                       # no entropy buffer
+    tra.tra_entropy = 8192
+    for field, bad in (("tra_tau", 0.0), ("tra_tau", float("nan")), ("tra_gamma", -0.5),
+                       ("tra_vote", 0)):
+        saved = getattr(tra, field)
+        setattr(tra, field, bad)
+        assert build(tra) == STA_ERR_ARG, field
+        setattr(tra, field, saved)
+    tra.kv_unit = 64
+    assert build(tra) == STA_ERR_UNSUPPORTED               # token lists are block_q wide
+    tra.kv_unit = 128
+    assert build(tra, Problem(1, 2000, 4, 4, 64, 0)) == STA_ERR_UNSUPPORTED  # > frame limit
+    assert lib.sta_build_blocks_rows(ctypes.byref(good), ctypes.byref(tra)) == 2 * 2
+    assert lib.sta_build_blocks_workspace(ctypes.byref(good), ctypes.byref(tra)) == 0
+
+    dyn = SelectorParams()
+    dyn.kind, dyn.block_q, dyn.kv_unit = STA_SEL_DYNRAD, 128, 128
+    dyn.radial_w0, dyn.radial_w_off, dyn.radial_full_df = 8, 1, 1
+    dyn.dyn_mode, dyn.dyn_ratio, dyn.dyn_threshold = 0, 0.35, 0.35
+    assert build(dyn, q=None) == STA_ERR_ARG               # needs q and k
+    assert build(dyn, Problem(2, 4, 8, 8, 64, 1)) == STA_ERR_UNSUPPORTED  # bf16 inputs only
+    for mode, ratio, thr in ((2, 0.35, 0.35), (0, 0.0, 0.35), (0, 1.5, 0.35),
+                             (1, 0.35, 0.0), (1, 0.35, float("nan"))):
+        dyn.dyn_mode, dyn.dyn_ratio, dyn.dyn_threshold = mode, ratio, thr
+        assert build(dyn) == STA_ERR_ARG, (mode, ratio, thr)
+    dyn.dyn_mode, dyn.dyn_ratio = 0, 1.0
+    dyn.kv_unit = 64
+    assert build(dyn) == STA_ERR_UNSUPPORTED
+    dyn.kv_unit = 128
+    # candidate limit: 1025 blocks of 128 tokens exceed the per-CTA candidate buffer
+    assert build(dyn, Problem(1, 1025, 8, 16, 64, 0)) == STA_ERR_UNSUPPORTED
+    ws = lib.sta_build_blocks_workspace(ctypes.byref(good), ctypes.byref(dyn))
+    # block means of q and k (fp32) and the prior lists fit in the workspace
+    assert ws >= 2 * 2 * 2 * 64 * 4 + 2 * 2 * 4 + 2 * 4
+    assert build(dyn) == STA_ERR_WORKSPACE                 # no workspace given
+    assert lib.sta_build_blocks_rows(ctypes.byref(good), ctypes.byref(dyn)) == 2 * 2
+
+    assert lib.sta_dense_attn_entropy_fwd(ctypes.byref(good), fake, fake, fake, 0.0, fake,
+                                          None, None, 0, None, None) == STA_ERR_ARG
+    assert lib.sta_dense_attn_entropy_fwd(ctypes.byref(Problem(1, 4, 8, 8, 96, 0)), fake, fake,
+                                          fake, 0.0, fake, fake, None, 0, None,
+                                          None) == STA_ERR_UNSUPPORTED
