@@ -5,19 +5,24 @@
 // static-ratio mode (speed first) and a dynamic-threshold mode (quality
 // first).  With the static radial list of query block b as its candidates:
 //
-//   s_c = scale * Qbar_b . Kbar_c     (block means, fp32, d summed in order)
+//   s_c = scale * Qbar_b . Kbar_c     (block means, fp32)
 //   p_c = softmax over the candidates of s_c
 //   rank: candidates ordered by s descending, ties to the lower block id
 //   static-ratio rho:      keep rank < k, k = ceil(rho * n * (1 - 1e-6)) in [1, n]
 //   dynamic-threshold th:  keep c iff the p mass of the ranks before c is
 //                          below th (the shortest prefix whose mass reaches th)
 //
-// One CTA per (query block, head).  The ranks come from a pairwise count
+// One CTA per (query block, head).  Each warp scores whole candidates: the
+// lanes split d (4 or 2 floats each, so one Kbar row is one coalesced 512- or
+// 256-byte read), four candidates are in flight per warp, and a butterfly
+// reduction leaves the dot product in every lane.  The ranks come from a pairwise count
 // (n <= kDynMaxCand candidates), the prefix masses from a double-precision
 // scan of p in rank order, and the kept ids, already in ascending block
 // order, are compacted with warp ballots and a block-wide scan.
 #include <cuda_runtime.h>
 #include <math.h>
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -44,6 +49,58 @@ struct DynArgs {
   int32_t* dev_status;
 };
 
+// Scores s_j of the n candidates into cand[] / sc[] (one warp per candidate).
+template <int D>
+__device__ __forceinline__ void dyn_scores(const DynArgs& a, const float* qb, const float* kh,
+                                           int b, int n, int* cand, float* sc) {
+  constexpr int V = D / 32;  // floats per lane: 4 (d = 128) or 2 (d = 64)
+  constexpr int U = 4;       // candidates in flight per warp
+  constexpr int kWarps = kDynThreads / 32;
+  using Vec = typename std::conditional<V == 4, float4, float2>::type;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Vec qv = __ldg(reinterpret_cast<const Vec*>(qb) + lane);
+  const int32_t* prow = a.prior_idx + static_cast<size_t>(b) * a.prior_cap;
+  for (int j0 = warp * U; j0 < n; j0 += kWarps * U) {
+    int c[U];
+    Vec kv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {  // j0 + u < n is the same in every lane
+      c[u] = 0;
+      kv[u] = Vec{};
+      if (j0 + u < n) {
+        c[u] = __ldg(prow + j0 + u);
+        kv[u] = __ldg(reinterpret_cast<const Vec*>(kh + static_cast<size_t>(c[u]) * D) + lane);
+      }
+    }
+    float acc[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      acc[u] = qv.x * kv[u].x;
+      acc[u] = fmaf(qv.y, kv[u].y, acc[u]);
+      if constexpr (V == 4) {
+        acc[u] = fmaf(qv.z, kv[u].z, acc[u]);
+        acc[u] = fmaf(qv.w, kv[u].w, acc[u]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int u = 0; u < U; ++u) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+    // lane u stores candidate j0 + u
+    float mine = acc[0];
+    int mc = c[0];
+#pragma unroll
+    for (int u = 1; u < U; ++u) {
+      mine = lane == u ? acc[u] : mine;
+      mc = lane == u ? c[u] : mc;
+    }
+    if (lane < U && j0 + lane < n) {
+      cand[j0 + lane] = mc;
+      sc[j0 + lane] = mine * a.scale;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kDynThreads) dynrad_lists_kernel(const DynArgs a) {
   __shared__ int cand[kDynMaxCand];
   __shared__ float sc[kDynMaxCand];
@@ -60,16 +117,13 @@ __global__ void __launch_bounds__(kDynThreads) dynrad_lists_kernel(const DynArgs
   const float* kh = a.kbar + static_cast<size_t>(head) * a.nb * a.d;
   if (threadIdx.x == 0) running = 0;
   // scores of the candidates
+  if (a.d == 128)
+    dyn_scores<128>(a, qb, kh, b, n, cand, sc);
+  else
+    dyn_scores<64>(a, qb, kh, b, n, cand, sc);
+  __syncthreads();
   float lmax = -INFINITY;
-  for (int j = threadIdx.x; j < n; j += kDynThreads) {
-    const int c = __ldg(a.prior_idx + static_cast<size_t>(b) * a.prior_cap + j);
-    cand[j] = c;
-    const float* kr = kh + static_cast<size_t>(c) * a.d;
-    float acc = 0.f;
-    for (int t = 0; t < a.d; ++t) acc = fmaf(__ldg(qb + t), __ldg(kr + t), acc);
-    sc[j] = acc * a.scale;
-    lmax = fmaxf(lmax, sc[j]);
-  }
+  for (int j = threadIdx.x; j < n; j += kDynThreads) lmax = fmaxf(lmax, sc[j]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
   if (lane == 0) red[warp] = lmax;

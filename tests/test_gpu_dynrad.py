@@ -51,11 +51,13 @@ def _check(w, L, q, k, heads, qblocks=None):
     return checked, near
 
 
+@pytest.mark.parametrize("d", [128, 64])
 @pytest.mark.parametrize("mode,param", [("static", 0.35), ("static", 0.8), ("dynamic", 0.35),
                                         ("dynamic", 0.9)])
-def test_small_grid_every_row(cuda_ok, mode, param):
-    # 6 x 10 x 26 = 1560 tokens: 13 blocks, the last one partial (24 tokens)
-    w = workload("dynrad_static", F=6, H=10, W=26, heads=2)
+def test_small_grid_every_row(cuda_ok, mode, param, d):
+    # 6 x 10 x 26 = 1560 tokens: 13 blocks, the last one partial (24 tokens);
+    # d = 128 and d = 64 take the 4- and 2-floats-per-lane score paths
+    w = workload("dynrad_static", F=6, H=10, W=26, heads=2, d=d)
     w["radial"] = dict(w0=260, w_off=1, full_df=-1)
     w["dynrad"] = dict(mode=mode, **({"ratio": param} if mode == "static" else
                                      {"threshold": param}))
