@@ -10,7 +10,8 @@ these pages:
 * "Token Radius Attention for Efficient Video Generation" (gist.science
   summary): dense 3D softmax attention (1. Problem Statement), block-level
   sparsity, per-query entropy and a radius neighbourhood (2. Methodology:
-  Insight I, Insight II, The TRA Pipeline).
+  Insight I, Insight II, The TRA Pipeline, including its tile-major token
+  layout).
 * "Radial Attention to Accelerate Video Generation" (blog): a static mask
   whose window shrinks with frame distance (The idea behind Radial Attention).
 * "Where Compute Matters: Heterogeneous Attention for Efficient Video
@@ -19,6 +20,9 @@ these pages:
 * "AB-Attention speeds up video diffusion transformers up to 2.23x, no
   training" (Glonce): intra-block clustering selector (IBCS), sampling with
   inclusion-probability weighting (SIP) (method paragraph, Key facts).
+* "DynamicRad: Content-Adaptive Sparse Attention for Long Video Diffusion":
+  static-ratio and dynamic-threshold selection inside a radial prior
+  (Abstract).
 
 Floating point is fp64 unless a page fixes the precision; inputs are the
 same bf16/fp32 values the library receives, widened exactly.  Library

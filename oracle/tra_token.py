@@ -93,21 +93,27 @@ def key_keep(i, H_i, F, Hh, W, tau, gamma):
     return kept, near
 
 
-def block_lists(H, F, Hh, W, B, tau, gamma, vote=1, qblocks=None):
+def block_lists(H, F, Hh, W, B, tau, gamma, vote=1, qblocks=None, perm=None):
     """Per query block: (ids, ambiguous) where ids are the key blocks kept
     when every pair is decided as stated (ascending) and ambiguous are the
     key blocks whose decision could change if near-threshold pairs went the
-    other way.  H: [N] entropies of one head."""
+    other way.  H: [N] entropies of one head, indexed by raster token.
+
+    perm (optional) is a token layout, perm[j] = raster token at sequence
+    position j (oracle/tile_major.py); blocks are then runs of B positions
+    of that sequence.  None is the raster layout."""
     N = F * Hh * W
     nb = n_blocks(N, B)
-    kb_of = np.arange(N) // B
+    perm = np.arange(N, dtype=np.int64) if perm is None else np.asarray(perm, dtype=np.int64)
+    kb_of = np.empty(N, np.int64)  # block of each raster token
+    kb_of[perm] = np.arange(N, dtype=np.int64) // B
     out = {}
     for qb in (range(nb) if qblocks is None else qblocks):
         lo, hi = block_range(qb, B, N)
         cnt = np.zeros(nb, np.int64)
         sure = np.zeros(nb, np.int64)
         maybe = np.zeros(nb, np.int64)
-        for i in range(lo, hi):
+        for i in perm[lo:hi]:
             kept, near = key_keep(i, H[i], F, Hh, W, tau, gamma)
             cnt += np.bincount(kb_of[kept], minlength=nb)
             sure += np.bincount(kb_of[kept & ~near], minlength=nb)
