@@ -196,10 +196,13 @@ int sta_build_blocks_rows(const sta_problem* prob, const sta_selector_params* se
 
 /*
  * Stage (a): selector.  q, k: device tensors [heads][N][d] (may be NULL for
- * the radial and routed kinds, which read only geometry / difficulty).
- * Writes `out` (see sta_block_lists).  Asynchronous on `stream`.
- * Errors: STA_ERR_ARG (null/inconsistent), STA_ERR_UNSUPPORTED (shape),
- * STA_ERR_WORKSPACE, STA_ERR_CUDA.
+ * the radial, routed and tra_token kinds, which read only geometry,
+ * difficulty or the entropies).  The kinds that read q and k (entropy,
+ * ibcs_sip, dynrad) take bf16 only.  Writes `out` (see sta_block_lists).
+ * Asynchronous on `stream`.
+ * Errors: STA_ERR_ARG (null/inconsistent, a parameter out of range),
+ * STA_ERR_UNSUPPORTED (shape, dtype or a size beyond a selector's limit),
+ * STA_ERR_WORKSPACE (workspace missing, short or misaligned), STA_ERR_CUDA.
  */
 sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* sel,
                             const void* q, const void* k, sta_block_lists* out,
