@@ -16,6 +16,9 @@ def _ptr(x):
     if isinstance(x, int):
         return x
     if isinstance(x, torch.Tensor):
+        # the library reads dense row-major buffers from the base pointer
+        if not x.is_contiguous():
+            raise ValueError("libsta takes contiguous tensors (got a strided view)")
         if x.device.type != "cuda":
             raise ValueError("libsta takes device tensors (got a host tensor)")
         return x.data_ptr()

@@ -138,3 +138,16 @@ def test_next_selector_argument_checks(lib):
     assert lib.sta_dense_attn_entropy_fwd(ctypes.byref(Problem(1, 4, 8, 8, 96, 0)), fake, fake,
                                           fake, 0.0, fake, fake, None, 0, None,
                                           None) == STA_ERR_UNSUPPORTED
+
+
+def test_binding_rejects_views_and_host_tensors():
+    import pytest
+    import torch
+    from sparse_spatiotemporal_attention_video_b200 import api
+    with pytest.raises(ValueError, match="contiguous"):
+        api._ptr(torch.zeros(4, 8).t())
+    with pytest.raises(ValueError, match="device"):
+        api._ptr(torch.zeros(4, 8))
+    with pytest.raises(TypeError):
+        api._ptr([1, 2])
+    assert api._ptr(None) is None and api._ptr(4096) == 4096
