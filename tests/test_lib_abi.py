@@ -151,3 +151,12 @@ def test_binding_rejects_views_and_host_tensors():
     with pytest.raises(TypeError):
         api._ptr([1, 2])
     assert api._ptr(None) is None and api._ptr(4096) == 4096
+
+
+def test_package_exports_every_selector_kind(lib):
+    import sparse_spatiotemporal_attention_video_b200 as pkg
+    from sparse_spatiotemporal_attention_video_b200 import _lib
+    kinds = [n for n in dir(_lib) if n.startswith("STA_SEL_")]
+    assert len(kinds) == 6
+    for n in kinds:
+        assert getattr(pkg, n) == getattr(_lib, n), n
