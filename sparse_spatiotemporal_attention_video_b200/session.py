@@ -44,12 +44,12 @@ def selector(w, difficulty=None, entropy=None):
         c = w["routed"]
         s.dense_frac, s.win_f, s.win_h, s.win_w = c["dense_frac"], c["win_f"], c["win_h"], c["win_w"]
         if difficulty is not None:
-            s.difficulty = difficulty.data_ptr()
+            s.difficulty = api._ptr(difficulty)
     elif w["selector"] == "tra_token":
         c = w["tra_token"]
         s.tra_tau, s.tra_gamma, s.tra_vote = c["tau"], c["gamma"], c["vote"]
         if entropy is not None:
-            s.tra_entropy = entropy.data_ptr()
+            s.tra_entropy = api._ptr(entropy)
     return s
 
 
