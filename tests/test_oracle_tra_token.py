@@ -5,6 +5,7 @@ and brute force on tiny grids."""
 import math
 
 import numpy as np
+import pytest
 
 from oracle import tra_token
 
@@ -141,3 +142,54 @@ def test_vote_above_pair_count_is_empty():
     H = np.ones(F * Hh * W)
     got = tra_token.block_lists(H, F, Hh, W, B, 1.0, 0.1, vote=10 ** 6)
     assert all(len(ids) == 0 for ids, _ in got.values())
+
+
+def _nearest_key_lists(H, F, Hh, W, B, tau, gamma):
+    """Vote-1 block lists from the nearest key of each grid-row segment: a
+    segment [w0, w1] of row (f, h) holds a kept key for query i iff its key
+    at column clamp(w_i, w0, w1) is kept (that key minimises the squared
+    distance within the row)."""
+    N = F * Hh * W
+    S = Hh * W
+    nb = (N + B - 1) // B
+    out = {}
+    for qb in range(nb):
+        kept = set()
+        for i in range(qb * B, min(N, qb * B + B)):
+            fi, hi, wi = i // S, (i % S) // W, i % W
+            r2 = tra_token.radius2(H[i], fi, F, tau, gamma)
+            for kb in range(nb):
+                if kb in kept:
+                    continue
+                t, t1 = kb * B, min(N, kb * B + B)
+                while t < t1:
+                    f, h, w0 = t // S, (t % S) // W, t % W
+                    w1 = min(W - 1, w0 + (t1 - 1 - t))
+                    t += w1 - w0 + 1
+                    if np.pi * r2[f] < 1.0:
+                        continue
+                    wn = min(max(wi, w0), w1)
+                    if (h - hi) ** 2 + (wn - wi) ** 2 <= r2[f]:
+                        kept.add(kb)
+                        break
+        out[qb] = sorted(kept)
+    return out
+
+
+@pytest.mark.parametrize("tau", [0.1, 0.15])
+@pytest.mark.parametrize("F,Hh,W,B,seed", [(3, 5, 7, 16, 0), (4, 6, 9, 32, 1), (2, 7, 5, 8, 2)])
+def test_vote_one_equals_nearest_key_of_each_row_segment(F, Hh, W, B, seed, tau):
+    # blocks straddle rows and frames (W and S are not multiples of B) and
+    # the last block is partial on the first two grids
+    N = F * Hh * W
+    H = np.random.default_rng(seed).uniform(1.0, 4.0, N)
+    gamma = 0.3
+    got = tra_token.block_lists(H, F, Hh, W, B, tau, gamma, vote=1)
+    ref = _nearest_key_lists(H, F, Hh, W, B, tau, gamma)
+    sizes = []
+    for qb, (ids, amb) in got.items():
+        assert len(amb) == 0
+        assert ids.tolist() == ref[qb], qb
+        sizes.append(len(ids))
+    nb = (N + B - 1) // B
+    assert 0 < min(sizes) and max(sizes) < nb  # neither empty nor dense rows
