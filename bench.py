@@ -375,7 +375,7 @@ def selector_bytes(w, lists_entries):
     if sel in ("entropy", "dynrad"):
         return 2 * h * N * d * 2 + 4 * lists_entries, "hbm"
     if sel == "ibcs_sip":
-        return 2 * h * N * d * 2 + 8 * lists_entries, "fma (fp32 importance GEMM)"
+        return 2 * h * N * d * 2 + 8 * lists_entries, "hbm (Q and K read once, lists written)"
     if sel == "routed":
         return 4 * N + 5 * N + 4 * lists_entries, "latency"
     if sel == "tra_token":

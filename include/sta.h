@@ -38,6 +38,8 @@
  *            Video Diffusion"
  *   [AB]    "AB-Attention speeds up video diffusion transformers up to 2.23x,
  *            no training"
+ *   [DYN]   "DynamicRad: Content-Adaptive Sparse Attention for Long Video
+ *            Diffusion"
  */
 #ifndef STA_H
 #define STA_H
@@ -195,7 +197,20 @@ size_t sta_build_blocks_workspace(const sta_problem* prob, const sta_selector_pa
 int sta_build_blocks_rows(const sta_problem* prob, const sta_selector_params* sel);
 
 /*
- * Stage (a): selector.  q, k: device tensors [heads][N][d] (may be NULL for
+ * Stage (a): selector.  Each kind restates one page's block selection:
+ *   STA_SEL_RADIAL    [RAD] The idea behind Radial Attention (static mask,
+ *                     window shrinking with frame distance);
+ *   STA_SEL_ENTROPY   [TRA] 2. Methodology, Insight I and The TRA Pipeline
+ *                     (entropy -> radius -> block mask), on pooled blocks;
+ *   STA_SEL_TRA_TOKEN [TRA] 2. Methodology, Insight II and The TRA Pipeline
+ *                     (budget tau*exp(H), decaying disks, token voting);
+ *   STA_SEL_IBCS_SIP  [AB] method paragraph (intra-block clustering
+ *                     importance, inclusion-probability sampling, 1/pi);
+ *   STA_SEL_ROUTED    [HETA] Abstract (uncertain tokens dense, rest local);
+ *   STA_SEL_DYNRAD    [DYN] Abstract (static-ratio / dynamic-threshold
+ *                     selection inside a radial prior).
+ * The formulas of each kind are in the sta_selector_params comment above.
+ * q, k: device tensors [heads][N][d] (may be NULL for
  * the radial, routed and tra_token kinds, which read only geometry,
  * difficulty or the entropies).  The kinds that read q and k (entropy,
  * ibcs_sip, dynrad) take bf16 only.  Writes `out` (see sta_block_lists).
@@ -282,7 +297,10 @@ sta_status sta_dense_attn_entropy_fwd(const sta_problem* prob, const void* q, co
  * until the process exits.
  * The first call on a device looks the array's device address up (with that
  * device current) and caches it; make that first call before any stream
- * capture.  Every call on every stream shares the one array and leaves its
+ * capture.  A reset of the device (cudaDeviceReset) unloads the array and
+ * leaves the cached address stale: do not use this entry point on a device
+ * after resetting it.  Argument errors (STA_ERR_ARG, STA_ERR_UNSUPPORTED)
+ * are checked before the size limit, as by sta_sparse_attn_fwd.  Every call on every stream shares the one array and leaves its
  * contents behind: two fp32 calls that may overlap on the GPU (different
  * streams, no ordering between them) race on it.  Calls on one stream are
  * ordered and safe.

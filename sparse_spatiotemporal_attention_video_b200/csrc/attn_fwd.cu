@@ -63,12 +63,7 @@ constexpr int kThreads = 352;
 constexpr int kHalfBytes = 128 * 128;  // 128 rows x 128 bytes: one 64-column half of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Tuning constants (compile-time).  One exponential pair in every
-// STA_POLY_EVERY pairs of a full tile goes to the FMA-pipe polynomial
-// (0 = all on MUFU); K/V ring depths.
-#ifndef STA_POLY_EVERY
-#define STA_POLY_EVERY 0
-#endif
+// Tuning constants (compile-time).
 // Deferred rescale: the running row maximum moves (and O is rescaled) only
 // when a tile's maximum exceeds it by more than this many log2 units.
 #ifndef STA_RESCALE_THRESHOLD
@@ -374,20 +369,9 @@ __device__ __forceinline__ float exp_store_half(const float (&x)[64], float scal
       const float o = off[c / W];
       const float2 arg = __ffma2_rn(make_float2(x[c], x[c + 1]), sl, make_float2(o, o));
       mx[i & 3] = fmax3(mx[i & 3], arg.x, arg.y);
-      float p0, p1;
-#if STA_POLY_EVERY > 0
-      if (simple && (i % STA_POLY_EVERY) == STA_POLY_EVERY - 1) {
-        p0 = exp2_poly(arg.x);
-        p1 = exp2_poly(arg.y);
-      } else {
-        p0 = fast_exp2(arg.x);
-        p1 = fast_exp2(arg.y);
-      }
-#else
       (void)simple;
-      p0 = fast_exp2(arg.x);
-      p1 = fast_exp2(arg.y);
-#endif
+      const float p0 = fast_exp2(arg.x);
+      const float p1 = fast_exp2(arg.y);
       pk[i] = pack_bf16x2(p0, p1);
       acc[i & 3] = __fadd2_rn(acc[i & 3], make_float2(bf16_lo(pk[i]), bf16_hi(pk[i])));
       if constexpr (ENT) {
@@ -480,7 +464,15 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
     const Item I = decode_item(a, it);
     int tok = -1;
     if (I.kind == kItemGatherDense) {
-      if (r < I.q_len) tok = __ldg(a.routed_ids + I.gbase + r);
+      // caller-supplied routed ids: an id outside [0, N) is skipped (its row
+      // neither read nor written) and reported
+      if (r < I.q_len) {
+        tok = __ldg(a.routed_ids + I.gbase + r);
+        if (tok < 0 || tok >= a.N) {
+          if (J == 0) raise_status(a.dev_status, STA_DEV_BAD_INDEX);
+          tok = -1;
+        }
+      }
     } else if (r < I.q_len) {
       tok = I.q_start + r;
     }
@@ -905,7 +897,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const __nv_bfloat16* qh = a.q + static_cast<size_t>(I.head) * a.N * D;
           for (int r = lane; r < kTileQ; r += 32) {
             const int src_r = (r < I.q_len) ? r : 0;
-            const int tok = __ldg(a.routed_ids + I.gbase + src_r);
+            int tok = __ldg(a.routed_ids + I.gbase + src_r);
+            // an out-of-range id (reported by the softmax warps, which skip
+            // its row) reads token 0 instead
+            if (tok < 0 || tok >= a.N) tok = 0;
             const uint4* src = reinterpret_cast<const uint4*>(qh + static_cast<size_t>(tok) * D);
 #pragma unroll
             for (int c = 0; c < D / 8; ++c) {

@@ -309,22 +309,4 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA/ALU pipes, for finite x >= -125 (the caller clamps; masked
-// -inf entries never take this path).  x = j + f with j = nearest integer
-// (obtained by adding 1.5*2^23, which leaves j in the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f is a cubic fitted by the Remez exchange algorithm on
-// relative error (coefficients from csrc/fit_exp2_poly.py; max relative
-// error 7.5e-5, far below the bf16 rounding of P); 2^j is added to the
-// exponent field: (bits(x + 1.5*2^23) << 23) == j << 23 modulo 2^32.
-__device__ __forceinline__ float exp2_poly(float x) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.999928057f, c1 = 0.693260968f, c2 = 0.242611125f, c3 = 0.0551716685f;
-  x = fmaxf(x, -125.0f);
-  const float t = __fadd_rn(x, kShift);
-  const float j = __fsub_rn(t, kShift);
-  const float f = __fsub_rn(x, j);
-  const float p = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, c0);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 }  // namespace sta

@@ -476,15 +476,33 @@ size_t sta_attn_workspace(const sta_problem* prob) {
   return prob->dtype == STA_F32 ? 3 * staged_bytes(prob) : 0;
 }
 
-sta_status sta_sparse_attn_fwd(const sta_problem* prob, const sta_attn_params* prm,
-                               const void* q, const void* k, const void* v,
-                               const sta_block_lists* lists, void* o, void* workspace,
-                               size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by the sparse attention entry points (before any
+// size or workspace check, so that both report the same codes).
+sta_status check_sparse_args(const sta_problem* prob, const sta_attn_params* prm, const void* q,
+                             const void* k, const void* v, const sta_block_lists* lists,
+                             const void* o) {
   sta_status st = check_problem(prob);
   if (st != STA_OK) return st;
   if (!prm || !q || !k || !v || !lists || !o) return STA_ERR_ARG;
   if (!pow2_unit(prm->block_q) || !pow2_unit(prm->kv_unit)) return STA_ERR_UNSUPPORTED;
   if (!lists->idx || !lists->cnt || lists->cap < 1) return STA_ERR_ARG;
+  return STA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sta_status sta_sparse_attn_fwd(const sta_problem* prob, const sta_attn_params* prm,
+                               const void* q, const void* k, const void* v,
+                               const sta_block_lists* lists, void* o, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  sta_status st = check_sparse_args(prob, prm, q, k, v, lists, o);
+  if (st != STA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int N = prob->F * prob->H * prob->W;
   AttnArgs a = {};
@@ -601,7 +619,10 @@ sta_status sta_dense_attn_entropy_fwd(const sta_problem* prob, const void* q, co
 // is used on holds kStaticStageBytes until the process exits.  Host code
 // cannot use the symbol's name as a device address (it names a host-side
 // shadow), so its device address is looked up once per device with
-// cudaGetSymbolAddress and cached.
+// cudaGetSymbolAddress and cached.  A reset of the device's primary context
+// (cudaDeviceReset) unloads the library's device image and makes the cached
+// address stale: this entry point must not be used on a device after such a
+// reset.
 namespace {
 
 constexpr size_t kStaticStageBytes = size_t(12) << 20;  // 12 MiB
@@ -635,7 +656,7 @@ extern "C" sta_status sta_sparse_attn_fwd_noalloc(const sta_problem* prob,
                                                   const void* k, const void* v,
                                                   const sta_block_lists* lists, void* o,
                                                   int32_t* dev_status, sta_stream_t stream) {
-  sta_status st = check_problem(prob);
+  sta_status st = check_sparse_args(prob, prm, q, k, v, lists, o);
   if (st != STA_OK) return st;
   if (prob->dtype != STA_F32) {
     // bf16 inputs feed the tensor cores directly: no scratch at all.

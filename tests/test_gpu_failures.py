@@ -1,7 +1,7 @@
 """Failure detection without a GPU fault: a bounded wait that runs out
 reports STA_DEV_TIMEOUT and leaves the context usable; list rows longer than
 their capacity are truncated, flagged and their true length reported; an
-out-of-range list entry is skipped and flagged."""
+out-of-range list entry or routed token id is skipped and flagged."""
 import numpy as np
 import pytest
 import torch
@@ -88,6 +88,42 @@ def test_out_of_range_entry_is_skipped_and_flagged(cuda_ok):
         lo, hi = qb * 128, min(w["N"], qb * 128 + 128)
         ref = block_sparse_rows(q[0], k[0], v[0], qb, units, 128, 32)
         assert_close_attn(oc[0, lo:hi].float().numpy(), ref, f"qb {qb}")
+
+
+def test_out_of_range_routed_id_is_skipped_and_flagged(cuda_ok):
+    """A routed id outside [0, N) in caller-written lists is neither read nor
+    written: its row is skipped, STA_DEV_BAD_INDEX is raised, and every other
+    row still equals the oracle."""
+    _lib, api, session = _mods()
+    from oracle.pipeline import routed_rows
+    from synthetic import make_difficulty
+    w = workload("heta_routed", heads=1, F=3, H=10, W=13)    # N = 390, 78 routed
+    q, k, v = make_qkv(w)
+    dif = make_difficulty(w)
+    L = session.Lists(w)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    api.sta_build_blocks(session.problem(w), session.selector(w, torch.from_numpy(dif).cuda()),
+                         None, None, L.struct, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    n = L.struct.n_routed
+    ids = L.routed_ids[:n].cpu().numpy().copy()
+    flag = L.routed_flag.cpu().numpy().astype(bool)
+    lost = ids[[3, n - 1]].copy()                 # these rows are skipped
+    L.routed_ids[3] = w["N"] + 7
+    L.routed_ids[n - 1] = -3
+    o = torch.full_like(q, float("nan"), device="cuda")
+    api.sta_sparse_attn_fwd(session.problem(w), session.attn_params(w), q.cuda(), k.cuda(),
+                            v.cuda(), L.struct, o, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & _lib.STA_DEV_BAD_INDEX
+    oc = o[0].cpu().float().numpy()
+    assert np.isnan(oc[lost]).all()               # skipped rows stay untouched
+    keep = np.setdiff1d(np.arange(w["N"]), lost)
+    c = w["routed"]
+    ref = routed_rows(q[0], k[0], v[0], keep, flag, w["F"], w["H"], w["W"], c["win_f"],
+                      c["win_h"], c["win_w"])
+    assert_close_attn(oc[keep], ref, "rows with valid ids")
 
 
 def test_misaligned_workspace_is_rejected(cuda_ok):
