@@ -39,7 +39,9 @@ recovered; importance sums to 1 and equals pure-Python loops on a tiny case;
 water filling meets sum(pi) = m, pi <= 1 and equals a bisection solve;
 frac = 1 keeps everything with weight 1 (dense result); the Monte-Carlo mean
 over seeds of the Horvitz-Thompson numerator and denominator approaches the
-dense values.
+dense values; the k-means margin (relative, floored at a squared distance of
+1, minimum over all iterations) equals hand values; near_draws flags exactly
+the draws within 1e-5 of pi.
 """
 import math
 
@@ -129,6 +131,15 @@ def sample(pi, seed, row):
     return np.nonzero(u < pi)[0].astype(np.int64), u
 
 
+def near_draws(u, pi):
+    """Sub-blocks whose keep decision u_j < pi_j lies within NEAR_THRESHOLD
+    of flipping (|u_j - pi_j| <= 1e-5): reported separately, since pi carries
+    the rounding of the importance."""
+    u = np.asarray(u, np.float64)
+    pi = np.asarray(pi, np.float64)
+    return np.nonzero(np.abs(u - pi) <= NEAR_THRESHOLD)[0]
+
+
 def select_row(qb, kbar, n_j, seed, row, k, iters, frac):
     """All steps for one (head, query block).
 
@@ -141,7 +152,7 @@ def select_row(qb, kbar, n_j, seed, row, k, iters, frac):
     m = target_count(frac, len(p))
     pi = water_fill(p, m)
     ids, u = sample(pi, seed, row)
-    near = np.nonzero(np.abs(u - pi) <= NEAR_THRESHOLD)[0]
+    near = near_draws(u, pi)
     return dict(ids=ids, logw=-np.log(pi[ids]), pi=pi, u=u, p=p,
                 margin=margin, near_ids=near, m=m)
 

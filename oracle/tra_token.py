@@ -31,10 +31,20 @@ Readings (the page prints no formulas beyond the two above):
    of the block pairs at the Wan shape, whatever the entropies.)
 5. Token voting: key block kb is kept for query block qb iff at least `vote`
    kept (i, j) pairs have i in qb and j in kb.
-Near-threshold pairs: |d^2 - r_f^2| <= NEAR * r_f^2 or |n_f - 1| <= NEAR
-(relative: r_f^2 and n_f carry the rounding of exp(H)).  A block whose
-decision depends on such pairs is reported separately (block_lists returns
-the ambiguous blocks).
+Near-threshold pairs: |d^2 - r_f^2| <= NEAR * r_f^2 or |n_f - 1| <= NEAR.
+A block whose decision depends on such pairs is reported separately
+(block_lists returns the ambiguous blocks).  NEAR = 2.5e-5 bounds the
+relative distance between an fp32 r_f^2 (or n_f) formed from an entropy
+within 2e-5 nats of this one and the fp64 value here:
+  * the entropy: |exp(H' - H) - 1| <= 2.0e-5;
+  * fp32 arithmetic, u = 2^-24 per rounding, 4u per expf (2 ulp): the
+    budget tau * expf(H) 6u (tau rounded to fp32, expf, product); G, a sum
+    of F expf terms in frame order, (F + 3)u; pi * G and the division 3u
+    (pi rounded, product, quotient); the decay expf and its product 5u; the
+    disk test's r_f^2 - dh^2 (dh^2 an exact integer) or the share
+    pi * r_f^2 2u: (F + 19)u in all, 2.4e-6 at F = 21 and below 5e-6 for
+    F <= 64.
+2.0e-5 + 5e-6 = 2.5e-5.
 
 Parity: pinned (tests/test_oracle_tra_token.py): entropy is ln N for equal
 logits and ~0 for one dominant logit and equals a pure-Python loop; gamma = 0
@@ -42,13 +52,15 @@ gives r0^2 = n / (pi F) and equal per-frame radii; the kept-key count of a
 query far from the frame edges equals the Gauss circle count; block lists
 equal a brute-force loop over all token pairs on tiny grids; a huge tau keeps
 every block, a tiny tau keeps nothing, and a steep decay keeps only the
-query's own frame; vote thresholds above the pair count give empty lists.
+query's own frame; vote thresholds above the pair count give empty lists;
+the near band flags a key at relative distance 1e-5 from the disk edge (or a
+share 1e-5 from one token) and not one at 4e-5.
 """
 import numpy as np
 
 from .grid import block_range, coords, n_blocks
 
-NEAR = 1e-4
+NEAR = 2.5e-5
 
 
 def query_entropy(q, k, scale):

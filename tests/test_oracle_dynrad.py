@@ -105,3 +105,35 @@ def test_select_stays_inside_the_radial_prior():
         got = dynrad.select(q, k, F, H, W, B, params, mode, **kw)
         for b, (ids, _) in got.items():
             assert set(ids) <= set(prior[b]) and len(ids) >= 1
+
+
+def test_static_near_flag_on_close_scores():
+    """Static ratio keeps 2 of 4; the kept-last and dropped-first candidates
+    are near when their probabilities differ by <= 1e-5 relative."""
+    cands = [10, 11, 12, 13]
+    for rel, near in ((0.5e-5, True), (2e-5, False)):
+        p = np.array([0.4, 0.3, 0.3 * (1 - rel), 0.1])
+        kept, flag = dynrad.select_row(p, cands, "static", rho=0.5)
+        assert kept == [10, 11] and bool(flag) == near, (rel, flag)
+
+
+def test_dynamic_near_flag_on_prefix_mass_and_close_scores():
+    cands = [3, 5, 8, 9]
+    # prefix mass 0.700004 reaches theta = 0.7 within 1e-5: near
+    kept, flag = dynrad.select_row(np.array([0.4, 0.3 + 4e-6, 0.2, 0.1]), cands, "dynamic",
+                                   theta=0.7)
+    assert kept == [3, 5] and flag
+    # 0.70003 is 3e-5 past theta, and the next candidate is far: not near
+    kept, flag = dynrad.select_row(np.array([0.4, 0.3 + 3e-5, 0.2, 0.1]), cands, "dynamic",
+                                   theta=0.7)
+    assert kept == [3, 5] and not flag
+    # a prefix 5e-6 short of theta is near too (one more rounding step and it
+    # would have stopped there)
+    kept, flag = dynrad.select_row(np.array([0.4, 0.3 - 5e-6, 0.2, 0.1]), cands, "dynamic",
+                                   theta=0.7)
+    assert kept == [3, 5, 8] and flag
+    # the last kept and the first dropped candidate within 1e-5 relative
+    for rel, near in ((0.5e-5, True), (2e-5, False)):
+        p = np.array([0.5, 0.3, 0.3 * (1 - rel), 0.05])
+        kept, flag = dynrad.select_row(p, cands, "dynamic", theta=0.75)
+        assert kept == [3, 5] and bool(flag) == near, (rel, flag)

@@ -108,3 +108,31 @@ def test_near_threshold_flags():
     alpha, beta = -1.0, 2.0           # thresholds at H* = 1.0 (t=1) and 1.5 (t=2)
     H = np.array([1.0 + 5e-6, 1.5 - 2e-6, 1.2, 1.0 + 2e-5])
     assert list(entropy.near_threshold(H, alpha, beta, 0, 2)) == [True, True, False, False]
+
+
+def test_calibrate_hand_worked():
+    """Entropies 0..9 (any order): with linear interpolation between order
+    statistics the 5th percentile is 0.45 and the 95th is 8.55.  Mapping them
+    to radius 1 and to the boundary of radius 3 (r_hi + 1 with r_hi = 2)
+    gives beta = 2 / 8.1 = 20/81 and alpha = 1 - 0.45 * 20/81 = 8/9, each
+    rounded to fp32."""
+    e = np.array([7.0, 2.0, 9.0, 0.0, 4.0, 1.0, 8.0, 3.0, 6.0, 5.0])
+    alpha, beta = entropy.calibrate(e, 1, 2)
+    assert alpha == float(np.float32(8.0 / 9.0))
+    assert beta == float(np.float32(20.0 / 81.0))
+
+
+def test_calibrate_maps_percentiles_to_the_radius_range():
+    rng = np.random.default_rng(4)
+    e = 5.4 + 0.1 * rng.random(3000)
+    for r_lo, r_hi in ((1, 2), (0, 3), (2, 6)):
+        alpha, beta = entropy.calibrate(e, r_lo, r_hi)
+        h5, h95 = np.percentile(e, 5), np.percentile(e, 95)
+        assert abs(alpha + beta * h5 - r_lo) <= 1e-5 * (1 + abs(alpha))
+        assert abs(alpha + beta * h95 - (r_hi + 1)) <= 1e-5 * (1 + abs(alpha))
+        r = entropy.radius(e, alpha, beta, r_lo, r_hi)
+        # the lowest 5% sit at r_lo, the top 5% are clamped at r_hi, and the
+        # middle spreads over every radius in between
+        assert set(np.unique(r).tolist()) == set(range(r_lo, r_hi + 1))
+        assert (r[e < h5 - 1e-6] == r_lo).all()
+        assert (r[e > h95 + 1e-6] == r_hi).all()

@@ -124,3 +124,53 @@ def test_horvitz_thompson_unbiased_over_seeds():
     # and the expected number kept is m
     kept = np.mean([len(ibcs_sip.sample(pi, sd, 0)[0]) for sd in range(2000)])
     assert abs(kept - 4.0) < 0.15
+
+
+def test_kmeans_margin_hand_values():
+    """The margin is min over queries and iterations of (d2nd - d1st) /
+    max(1, d1st), squared L2 distances.  1-D points, k = 2, initial centroids
+    q[0] and q[2].
+
+    Points 0, 4, 10, 20 with centroids 0 and 10: the distance pairs are
+    (0, 100), (16, 36), (100, 0), (400, 100), so the margins are 100, 20/16,
+    100 and 300/100; the minimum is 1.25 (an absolute margin would give 20).
+    The second iteration (centroids 2 and 15) gives 29.25, 55.25, 1.56 and
+    11.96, so the minimum over both iterations stays 1.25."""
+    q = np.array([[0.0], [4.0], [10.0], [20.0]])
+    for iters in (1, 2):
+        _, _, margin = ibcs_sip.kmeans(q, 2, iters)
+        assert abs(margin - 1.25) <= 1e-15, (iters, margin)
+    # below a squared distance of 1 the margin is absolute: points 0, 0.3,
+    # 0.8, 5 (centroids 0 and 0.8) give pairs (0, .64), (.09, .25), (.64, 0),
+    # (25, 17.64): margins .64, .16, .64 and 7.36/17.64; a purely relative
+    # margin would give .16/.09 for the second point
+    q = np.array([[0.0], [0.3], [0.8], [5.0]])
+    _, _, margin = ibcs_sip.kmeans(q, 2, 1)
+    assert abs(margin - 0.16) <= 1e-15, margin
+
+
+def test_kmeans_margin_uses_the_two_nearest_of_four():
+    """With k = 4 the margin compares the two smallest of the four distances.
+    2-D points; the initial centroids are the points at offsets 0, 1, 2, 3
+    (n_b = 4): every point is its own centroid, so the smallest distance is 0
+    and each margin is the (floored) distance to its nearest other point."""
+    q = np.array([[0.0, 0.0], [3.0, 0.0], [0.0, 10.0], [3.0, 12.0]])
+    # nearest-other squared distances: 9, 9, 13, 13 -> margin 9
+    _, counts, margin = ibcs_sip.kmeans(q, 4, 1)
+    assert list(counts) == [1, 1, 1, 1]
+    assert margin == 9.0
+
+
+def test_near_draws_band():
+    pi = np.array([0.3, 0.3, 0.3, 0.3, 0.7, 1.0, 0.05])
+    u = np.array([0.3 + 5e-6, 0.3 - 5e-6, 0.3 + 2e-5, 0.3 - 2e-5, 0.7, 0.999995, 0.9])
+    assert ibcs_sip.near_draws(u, pi).tolist() == [0, 1, 4, 5]
+
+
+def test_select_row_reports_its_near_draws():
+    rng = np.random.default_rng(5)
+    qb = rng.normal(size=(128, 16))
+    kbar, n_j = ibcs_sip.subblock_means(rng.normal(size=(512, 16)), 16)
+    row = ibcs_sip.select_row(qb, kbar, n_j, 7, 3, 4, 5, 0.25)
+    assert row["near_ids"].tolist() == ibcs_sip.near_draws(row["u"], row["pi"]).tolist()
+    assert row["ids"].tolist() == np.nonzero(row["u"] < row["pi"])[0].tolist()

@@ -193,3 +193,35 @@ def test_vote_one_equals_nearest_key_of_each_row_segment(F, Hh, W, B, seed, tau)
         sizes.append(len(ids))
     nb = (N + B - 1) // B
     assert 0 < min(sizes) and max(sizes) < nb  # neither empty nor dense rows
+
+
+@pytest.mark.parametrize("delta,near", [(1e-5, True), (-1e-5, True), (4e-5, False),
+                                        (-4e-5, False)])
+def test_near_band_at_the_disk_edge(delta, near):
+    """One frame (G = 1, no decay), H = 0: r^2 = tau / pi.  With
+    tau = 25 pi (1 + delta) the key at (dh, dw) = (3, 4) sits at d^2 = 25, a
+    relative distance |delta| / (1 + delta) from the disk edge: near within
+    2.5e-5, kept iff delta >= 0."""
+    F, Hh, W = 1, 11, 11
+    i = 5 * W + 5                                   # the centre token
+    tau = 25.0 * math.pi * (1.0 + delta)
+    kept, nr = tra_token.key_keep(i, 0.0, F, Hh, W, tau, 0.25)
+    j = (5 + 3) * W + (5 + 4)
+    assert bool(kept[j]) == (delta > 0)
+    assert bool(nr[j]) == near
+    # keys one unit of d^2 away are far from the edge
+    for j2 in ((5 + 5) * W + 5 - 1, 5 * W + 5 + 4):  # d^2 = 26 and 16
+        assert not nr[j2]
+
+
+@pytest.mark.parametrize("delta,near", [(1e-5, True), (-1e-5, True), (4e-5, False),
+                                        (-4e-5, False)])
+def test_near_band_at_one_token_share(delta, near):
+    """One frame, H = 0, tau = 1 + delta: the frame's share is n_f = tau
+    tokens.  The query's own key (d^2 = 0, far inside the disk) is kept iff
+    n_f >= 1, and near iff n_f is within 2.5e-5 of one token."""
+    F, Hh, W = 1, 5, 5
+    i = 12
+    kept, nr = tra_token.key_keep(i, 0.0, F, Hh, W, 1.0 + delta, 0.25)
+    assert bool(kept[i]) == (delta > 0)
+    assert bool(nr[i]) == near
