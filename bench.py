@@ -1,11 +1,18 @@
 """Benchmark: one step of the sparse-attention hot path on B200.
 
-Default workload: static radial sparse attention at the Wan2.1-1.3B latent
-grid (12 heads x 21x30x52 = 32,760 tokens x d=128, bf16, 128-token blocks).
-One step = the selector (sta_build_blocks) plus the block-sparse attention
+Default workload: importance-sampled block attention at the HunyuanVideo
+latent grid (24 heads x 33x45x80 = 118,800 tokens x d=128, bf16, 128-query
+blocks, 16-key sub-blocks, ~10% sampled), the largest workload that fits one
+GPU.  One step = the selector (sta_build_blocks: sub-block means, k-means,
+importance, Philox sampling) plus the weighted block-sparse attention
 (sta_sparse_attn_fwd) on one batch.  --workload picks the other workloads
-(tra_entropy, heta_routed, ab_sampled); a step is then that workload's
-selector plus attention.
+(wan_radial, tra_entropy, heta_routed, tra_token, dynrad_static,
+dynrad_dynamic); a step is then that workload's selector plus attention.
+
+Timing: the step, selector-only and attention-only CUDA graphs are replayed
+in one interleaved loop, each after the same L2 flush, so the three device
+times come from the same clock state; every figure is a mean over the K
+timed iterations.
 
 Reported (one JSON line on rank 0):
   value      effective TFLOP/s on retained blocks (4*d FLOPs per kept
@@ -39,7 +46,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "effective TFLOP/s on retained blocks; speedup vs dense at same shape (1×B200)"
-DEFAULT_WORKLOAD = "wan_radial"
+DEFAULT_WORKLOAD = "ab_sampled"
 WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled", "tra_token",
              "dynrad_static", "dynrad_dynamic")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -363,7 +370,7 @@ def config_of(w):
 
 
 # ------------------------------------------------------------------- GPU arm
-SELECTOR_LAUNCHES = {"radial": 1, "entropy": 2, "routed": 2, "ibcs_sip": 5, "tra_token": 1,
+SELECTOR_LAUNCHES = {"radial": 1, "entropy": 3, "routed": 2, "ibcs_sip": 6, "tra_token": 1,
                      "dynrad": 3}
 
 
@@ -486,14 +493,30 @@ def main(argv=None):
         torch.cuda.synchronize()
         return [a.elapsed_time(b) for a, b in ts]
 
+    # K iterations of (step, selector alone, attention alone), interleaved,
+    # each replay after the same L2 flush and timed with its own events on
+    # the launching stream
+    run_sel = graphs["select"].replay if graphs else select
+    run_att = graphs["attend"].replay if graphs else attend
     barrier(ws)
     with ClockSampler(local) as clk:
-        step_ms = timed(run_step, args.steps)
+        ev = []
+        for _ in range(args.steps):
+            trip = []
+            for fn in (run_step, run_sel, run_att):
+                l2_flush.zero_()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                fn()
+                b.record()
+                trip.append((a, b))
+            ev.append(trip)
+        torch.cuda.synchronize()
     barrier(ws)
+    step_ms = [t[0][0].elapsed_time(t[0][1]) for t in ev]
+    sel_ms = [t[1][0].elapsed_time(t[1][1]) for t in ev]
+    attn_ms = [t[2][0].elapsed_time(t[2][1]) for t in ev]
     ms = max_over_ranks(sum(step_ms) / len(step_ms), ws)
-    n_stage = max(5, min(20, args.steps))
-    sel_ms = timed(graphs["select"].replay if graphs else select, n_stage)
-    attn_ms = timed(graphs["attend"].replay if graphs else attend, n_stage)
     sel_avg = sum(sel_ms) / len(sel_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
 
@@ -542,9 +565,13 @@ def main(argv=None):
         "metric": METRIC, "value": total_flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": dict(config_of(w), cuda_graph=bool(graphs)),
+        "data": "synthetic", "config": config_of(w), "cuda_graph": bool(graphs),
         "retained_pairs": pairs, "retained_fraction": pairs / (w["N"] ** 2 * w["heads"]),
-        "attn_ms": attn_avg, "dense_ms": dense_avg,
+        "attn_ms": attn_avg, "selector_ms": sel_avg,
+        "stage_medians_ms": {"step": sorted(step_ms)[len(step_ms) // 2],
+                             "selector": sorted(sel_ms)[len(sel_ms) // 2],
+                             "attention": sorted(attn_ms)[len(attn_ms) // 2]},
+        "dense_ms": dense_avg,
         "dense_tflops": dense_flops / (dense_avg * 1e-3) / 1e12,
         "speedup_vs_dense": dense_avg / attn_avg,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

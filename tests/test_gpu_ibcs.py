@@ -73,19 +73,58 @@ def test_ibcs_small_grids_every_row(cuda_ok, F, H, W, frac):
     assert checked >= 1 and skipped <= 1 and near <= 2
 
 
-def test_ibcs_full_hunyuan_shape_sampled_rows(cuda_ok):
+@pytest.fixture(scope="module")
+def hunyuan(cuda_ok):
+    """The full HunyuanVideo-shape workload (24 heads x 33x45x80 tokens x 128,
+    bf16) on the device with its GPU lists, shared by the full-size tests."""
     w = workload("ab_sampled")
-    q, k, _ = make_qkv(w)
-    L = _gpu_select(w, q.cuda(), k.cuda())
+    q, k, v = make_qkv(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    L = _gpu_select(w, qd, kd)
     nqb = (w["N"] + 127) // 128
     rng = np.random.default_rng(2)
-    qblocks = [0, nqb - 1] + sorted(rng.choice(nqb - 2, 6, replace=False) + 1)
+    qblocks = [0, nqb - 1] + sorted((rng.choice(nqb - 2, 6, replace=False) + 1).tolist())
+    yield dict(w=w, q=q, k=k, v=v, qd=qd, kd=kd, vd=vd, L=L, qblocks=qblocks)
+    del qd, kd, vd
+    torch.cuda.empty_cache()
+
+
+def test_ibcs_full_hunyuan_shape_sampled_rows(hunyuan):
+    w, q, k, L, qblocks = (hunyuan[x] for x in ("w", "q", "k", "L", "qblocks"))
     checked, skipped, near = _check_rows(w, L, q, k, (0, 13, 23), qblocks)
     assert checked >= 20 and skipped <= 2 and near <= 4
     # about 10% of the sub-blocks are kept per row
     m = ibcs_sip.target_count(w["ibcs"]["sample_frac"], (w["N"] + 15) // 16)
     cnt = L.cnt.cpu().numpy()
     assert abs(cnt.mean() - m) < 3.0, (cnt.mean(), m)
+
+
+def test_weighted_attention_full_hunyuan_shape_sampled_blocks(hunyuan):
+    """SIP-weighted attention at the full HunyuanVideo shape: about 743 sampled
+    16-key units (93 tiles) per query block, log-weights up to ln(1/pi_min).
+    The GPU output of the first, last and 6 seeded query blocks of heads 0,
+    13 and 23 against the oracle over the same lists and weights."""
+    api, session = _lib()
+    w, q, k, v, L, qblocks = (hunyuan[x] for x in ("w", "q", "k", "v", "L", "qblocks"))
+    o = torch.full_like(hunyuan["qd"], float("nan"))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    api.sta_sparse_attn_fwd(session.problem(w), session.attn_params(w), hunyuan["qd"],
+                            hunyuan["kd"], hunyuan["vd"], L.struct, o, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0, api.sta_dev_status_string(int(st.item()))
+    N = w["N"]
+    nqb = (N + 127) // 128
+    cnt = L.cnt.cpu().numpy()
+    idx = L.idx.cpu().numpy()
+    lw = L.logw.cpu().numpy()
+    assert float(lw[cnt > 0].max()) > 1.0  # weights well away from 1 are exercised
+    for h in (0, 13, 23):
+        for qb in qblocks:
+            r = h * nqb + qb
+            units = idx[r, :cnt[r]].tolist()
+            ref = block_sparse_rows(q[h], k[h], v[h], qb, units, 128, 16, lw[r, :cnt[r]])
+            lo, hi = qb * 128, min(N, qb * 128 + 128)
+            assert_close_attn(o[h, lo:hi].float().cpu().numpy(), ref, f"head {h} qb {qb}")
 
 
 def test_sampled_attention_matches_oracle(cuda_ok):
