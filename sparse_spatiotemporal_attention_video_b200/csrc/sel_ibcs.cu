@@ -43,25 +43,23 @@ namespace sta {
 namespace {
 
 // ------------------------------------------------------------------ k-means
-// One CTA of 256 threads per (head, query block), the block staged once in
-// shared memory as bf16 (exact) and its fp32 values held in registers.
+// One CTA of 128 threads per (head, query block); thread r owns query r.
 //
-// Assignment: thread (g, p) = (tid / 64, tid % 64) owns queries p and p + 64
-// over dimension quarter g (32 fp32 values each, in registers for all
-// iterations) and forms the partial squared distances to every centroid
-// with packed f32x2 subtract / fused multiply-add (even and odd dimensions
-// in the two halves, added at the end); the centroids are read from shared
-// memory as warp-uniform 16-byte broadcasts.  The four quarter partials of a
-// query are added in order g = 0..3 and the argmin keeps the lower index on
-// ties.  The direct form sum (x - c)^2 is kept (not |c|^2 - 2 x.c): it has no
-// cancellation, so the distance carries fp32 rounding relative to itself.
-//
-// Update: the members are counting-sorted by cluster (warp ballots), so the
-// member sum of dimension pair j over cluster c is a run of plain adds; thread
-// (s, j) = (tid / 64, tid % 64) sums dimension pair j over the quarter s of
-// the sorted members, cut at cluster boundaries, and the four partials are
-// added in order.  An empty cluster keeps its centroid.
-constexpr int kKmThreads = 256;
+// The block is staged once in shared memory as bf16 (exact), with a row
+// pitch that makes each thread's 8-byte reads of its own row conflict-free.
+// Assignment: thread r forms the squared distances to every centroid over
+// the 128 dimensions itself (packed f32x2 subtract / fused multiply-add,
+// even and odd dimensions in the two halves, added at the end; centroids are
+// warp-uniform shared-memory broadcasts) and takes the argmin, ties to the
+// lower index.  The direct form sum (x - c)^2 is kept (not |c|^2 - 2 x.c):
+// it has no cancellation, so a distance carries fp32 rounding relative to
+// itself.
+// Update: the members are counting-sorted by cluster (warp ballots), then
+// thread t sums dimension pair t % 64 over the members of clusters
+// t / 64, t / 64 + 2, ... in sorted order (runs of plain adds) and writes the
+// mean.  An empty cluster keeps its centroid.  Three barriers per iteration.
+constexpr int kKmThreads = 128;
+constexpr int kKmWarps = kKmThreads / 32;
 constexpr int kKmRows = 128;           // largest query block
 constexpr int kKmRowPitch = 128 + 8;   // bf16 per staged row (272 B: conflict-free 16 B reads)
 
@@ -69,14 +67,13 @@ template <int KM>
 struct KmSmem {
   __nv_bfloat16 q[kKmRows * kKmRowPitch];  // staged block, rows >= nb zero
   float negc[KM * 128];                    // -centroid
-  float part[4 * KM * kKmRows];            // [g][c][r] distances / [s][c][dim] sums
   int perm[kKmRows];                       // members sorted by cluster
-  int wcount[4][KM];                       // per-warp member counts (warps 0-3)
+  int wcount[kKmWarps][KM];                // per-warp member counts
   int start[KM + 1];                       // first sorted position of each cluster
 };
 
 template <int KM>
-__global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 1 : 2) kmeans_kernel(
+__global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 4 : 6) kmeans_kernel(
     const __nv_bfloat16* __restrict__ q, int N, int B, int nqb, int iters,
     float* __restrict__ cent, float* __restrict__ wts) {
   constexpr int D = 128;
@@ -103,65 +100,37 @@ __global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 1 : 2) kmeans_kernel(
     const int c = i / D, col = i - c * D;
     sm.negc[i] = -__bfloat162float(sm.q[((c * nb) / KM) * kKmRowPitch + col]);
   }
-  // registers: queries p and p + 64, dimensions [32g, 32g + 32) as 16 pairs
-  const int g = tid >> 6, p = tid & 63;
-  float2 x[2][16];
-#pragma unroll
-  for (int qi = 0; qi < 2; ++qi) {
-#pragma unroll
-    for (int v8 = 0; v8 < 4; ++v8) {
-      const uint4 w =
-          *reinterpret_cast<const uint4*>(&sm.q[(p + 64 * qi) * kKmRowPitch + 32 * g + 8 * v8]);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int t = 0; t < 4; ++t)
-        x[qi][4 * v8 + t] = make_float2(__uint_as_float(ww[t] << 16),
-                                        __uint_as_float(ww[t] & 0xffff0000u));
-    }
-  }
   __syncthreads();
+  const __nv_bfloat16* xrow = &sm.q[tid * kKmRowPitch];  // this thread's query
 
   for (int it = 0; it < iters; ++it) {
-    // ---- assignment: partial distances over quarter g
+    // ---- assignment (thread = query) and per-warp cluster counts
+    int best = -1, rank = 0;
     {
-      float2 acc[2][KM];
+      float2 acc[KM];
 #pragma unroll
-      for (int qi = 0; qi < 2; ++qi)
+      for (int c = 0; c < KM; ++c) acc[c] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int c = 0; c < KM; ++c) acc[qi][c] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int j4 = 0; j4 < D / 4; ++j4) {  // 4 dimensions per step
+        const uint2 w = *reinterpret_cast<const uint2*>(xrow + 4 * j4);
+        const float2 x0 = make_float2(__uint_as_float(w.x << 16),
+                                      __uint_as_float(w.x & 0xffff0000u));
+        const float2 x1 = make_float2(__uint_as_float(w.y << 16),
+                                      __uint_as_float(w.y & 0xffff0000u));
 #pragma unroll
         for (int c = 0; c < KM; ++c) {
-          const float4 nc = *reinterpret_cast<const float4*>(&sm.negc[c * D + 32 * g + 4 * i]);
-          const float2 n0 = make_float2(nc.x, nc.y), n1 = make_float2(nc.z, nc.w);
-#pragma unroll
-          for (int qi = 0; qi < 2; ++qi) {
-            const float2 t0 = __fadd2_rn(x[qi][2 * i], n0);
-            acc[qi][c] = __ffma2_rn(t0, t0, acc[qi][c]);
-            const float2 t1 = __fadd2_rn(x[qi][2 * i + 1], n1);
-            acc[qi][c] = __ffma2_rn(t1, t1, acc[qi][c]);
-          }
+          const float4 nc = *reinterpret_cast<const float4*>(&sm.negc[c * D + 4 * j4]);
+          const float2 t0 = __fadd2_rn(x0, make_float2(nc.x, nc.y));
+          acc[c] = __ffma2_rn(t0, t0, acc[c]);
+          const float2 t1 = __fadd2_rn(x1, make_float2(nc.z, nc.w));
+          acc[c] = __ffma2_rn(t1, t1, acc[c]);
         }
       }
-#pragma unroll
-      for (int qi = 0; qi < 2; ++qi)
-#pragma unroll
-        for (int c = 0; c < KM; ++c)
-          sm.part[(g * KM + c) * kKmRows + p + 64 * qi] = acc[qi][c].x + acc[qi][c].y;
-    }
-    __syncthreads();
-    // ---- argmin and counting sort (warps 0-3: thread r = query r)
-    int best = -1, rank = 0;
-    if (tid < kKmRows) {
-      const int r = tid;
-      if (r < nb) {
+      if (tid < nb) {
         float bd = 0.f;
 #pragma unroll
         for (int c = 0; c < KM; ++c) {
-          float d = sm.part[c * kKmRows + r];
-#pragma unroll
-          for (int gg = 1; gg < 4; ++gg) d += sm.part[(gg * KM + c) * kKmRows + r];
+          const float d = acc[c].x + acc[c].y;
           if (c == 0 || d < bd) {
             bd = d;
             best = c;
@@ -176,50 +145,41 @@ __global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 1 : 2) kmeans_kernel(
       }
     }
     __syncthreads();
-    if (tid < kKmRows) {
-      if (best >= 0) {
-        int pos = rank;
-        for (int c = 0; c < best; ++c)
+    // ---- counting sort: members of cluster 0, then 1, ...
+    if (best >= 0) {
+      int pos = rank;
+      for (int c = 0; c < best; ++c)
 #pragma unroll
-          for (int w = 0; w < 4; ++w) pos += sm.wcount[w][c];
-        for (int w = 0; w < warp; ++w) pos += sm.wcount[w][best];
-        sm.perm[pos] = tid;
-      }
-      if (tid <= KM) {
-        int s0 = 0;
-        for (int c = 0; c < tid; ++c)
+        for (int w = 0; w < kKmWarps; ++w) pos += sm.wcount[w][c];
+      for (int w = 0; w < warp; ++w) pos += sm.wcount[w][best];
+      sm.perm[pos] = tid;
+    }
+    if (tid <= KM) {
+      int s0 = 0;
+      for (int c = 0; c < tid; ++c)
 #pragma unroll
-          for (int w = 0; w < 4; ++w) s0 += sm.wcount[w][c];
-        sm.start[tid] = s0;
-      }
+        for (int w = 0; w < kKmWarps; ++w) s0 += sm.wcount[w][c];
+      sm.start[tid] = s0;
     }
     __syncthreads();
-    // ---- update: member sums of dimension pair j over sorted quarter s
+    // ---- update: mean of the members, dimension pair j of cluster c
     {
-      const int s = tid >> 6, j = tid & 63;
-      const int lo = (s * nb) >> 2, hi = ((s + 1) * nb) >> 2;
+      const int j = tid & 63;
 #pragma unroll
-      for (int c = 0; c < KM; ++c) {
-        const int a = max(lo, sm.start[c]), b = min(hi, sm.start[c + 1]);
-        float2 acc = make_float2(0.f, 0.f);
-        for (int t = a; t < b; ++t) {
-          const uint32_t w =
-              *reinterpret_cast<const uint32_t*>(&sm.q[sm.perm[t] * kKmRowPitch + 2 * j]);
-          acc = __fadd2_rn(acc, make_float2(__uint_as_float(w << 16),
-                                            __uint_as_float(w & 0xffff0000u)));
+      for (int c = tid >> 6; c < KM; c += kKmThreads / 64) {
+        const int a = sm.start[c], b = sm.start[c + 1];
+        if (b > a) {
+          float2 acc = make_float2(0.f, 0.f);
+          for (int t = a; t < b; ++t) {
+            const uint32_t w =
+                *reinterpret_cast<const uint32_t*>(&sm.q[sm.perm[t] * kKmRowPitch + 2 * j]);
+            acc = __fadd2_rn(acc, make_float2(__uint_as_float(w << 16),
+                                              __uint_as_float(w & 0xffff0000u)));
+          }
+          const float n = static_cast<float>(b - a);
+          *reinterpret_cast<float2*>(&sm.negc[c * D + 2 * j]) = make_float2(-(acc.x / n),
+                                                                            -(acc.y / n));
         }
-        *reinterpret_cast<float2*>(&sm.part[(s * KM + c) * D + 2 * j]) = acc;
-      }
-    }
-    __syncthreads();
-    for (int i = tid; i < KM * D; i += kKmThreads) {
-      const int c = i / D, col = i - c * D;
-      const int n = sm.start[c + 1] - sm.start[c];
-      if (n > 0) {
-        float acc = sm.part[c * D + col];
-#pragma unroll
-        for (int s = 1; s < 4; ++s) acc += sm.part[(s * KM + c) * D + col];
-        sm.negc[i] = -(acc / static_cast<float>(n));
       }
     }
     __syncthreads();
@@ -292,114 +252,196 @@ __device__ __forceinline__ void philox4x32_10_x2(uint4& a, uint4& b, uint32_t k0
   }
 }
 
-// One CTA per (head, query block) row of p.  Shared memory: p of the row
-// (ld = n_sub rounded up to 4 floats) and one flag byte per sub-block
-// (bit 0 capped, bit 1 kept).
+// Sum of an int and a double over the CTA with one barrier: the partials go
+// to slot `slot` of double-buffered shared arrays, so that consecutive calls
+// alternate slots and a slot is rewritten only after every thread has passed
+// the barrier of the call in between.
+__device__ __forceinline__ void block_sum2(int& c, double& d, int slot, int (*rc)[kSipWarps],
+                                           double (*rd)[kSipWarps]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+    d += __shfl_xor_sync(0xffffffffu, d, o);
+  }
+  if (lane == 0) {
+    rc[slot][warp] = c;
+    rd[slot][warp] = d;
+  }
+  __syncthreads();
+  c = 0;
+  d = 0.0;
+#pragma unroll
+  for (int w = 0; w < kSipWarps; ++w) {
+    c += rc[slot][w];
+    d += rd[slot][w];
+  }
+}
+
+// One CTA per (head, query block) row of p.  Thread t owns the Philox groups
+// (4 consecutive sub-blocks each) t, t + T, ..., t + (G-1) T and keeps their
+// p in registers for every pass:
 //  - Water filling: each round caps every uncapped j with lambda p_j >= 1
-//    and, in the same pass, sums (fp64) the p of the sub-blocks that stay
-//    uncapped, which is the next round's denominator.
-//  - Draws: thread t takes the Philox groups t, t + T, ... two at a time and
-//    sets the kept bit where u_j < pi_j; pi_j = 1 for capped j, else
-//    min(1, lambda p_j) in fp64.
-//  - Output: thread t owns a contiguous chunk of sub-blocks (a multiple of 4),
-//    counts its kept bits, and an exclusive block scan places its ids in
-//    ascending order, with logw = -ln pi.
-__global__ void __launch_bounds__(kSipThreads) sip_sample_kernel(
+//    and, in the same pass, sums the p of the sub-blocks that stay uncapped,
+//    the next round's denominator; one barrier per round.
+//  - Draws: one Philox block per group (two groups in lockstep); j is kept
+//    where u_j < pi_j, with pi_j = 1 for capped j, else min(1, lambda p_j).
+//  - Output: ids in ascending order are groups in (k, t) order; an exclusive
+//    block scan of the per-group kept counts over t, offset by the totals of
+//    the earlier k, places them; logw = -ln pi.
+// Precision: lambda and the sums across threads are fp64; a thread's own
+// sums are pairwise in fp32 (relative error ~3e-7), and the per-element
+// comparisons use lambda rounded to fp32.  A decision can then differ from
+// an fp64 evaluation only where lambda p_j or u_j lies within ~1e-6 of the
+// threshold, inside the 1e-5 band in which sampling decisions are reported
+// as near-threshold; a cap decision that differs there moves pi_j by less
+// than 1e-6 and lambda by far less.
+template <int G>
+__global__ void __launch_bounds__(kSipThreads, G <= 8 ? 4 : 1) sip_sample_kernel(
     const float* __restrict__ p, int n_sub, int m, uint32_t seed_lo, uint32_t seed_hi,
     int32_t* __restrict__ idx, float* __restrict__ logw, int32_t* __restrict__ cnt, int cap,
     int32_t* required_cap, int32_t* dev_status) {
-  extern __shared__ __align__(16) float sip_smem[];
-  const int ld = (n_sub + 3) & ~3;
-  float* sp = sip_smem;                                          // [ld]
-  uint8_t* flag = reinterpret_cast<uint8_t*>(sp + ld);           // [ld]
-  __shared__ double redd[kSipWarps];
-  __shared__ int redi[kSipWarps];
-  const int tid = threadIdx.x;
+  constexpr int MW = (4 * G + 31) / 32;  // words of the per-thread bit masks
+  __shared__ int rc[2][kSipWarps];
+  __shared__ double rd[2][kSipWarps];
+  __shared__ int tab[kSipWarps][G];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.x;  // head * nqb + qb
+  const int ld = (n_sub + 3) & ~3;
+  const int n_grp = ld / 4;
   const float4* pr = reinterpret_cast<const float4*>(p + static_cast<size_t>(row) * ld);
-  double part = 0.0;
-  for (int i = tid; i < ld / 4; i += kSipThreads) {
-    const float4 v = __ldcs(pr + i);  // padding columns hold 0
-    reinterpret_cast<float4*>(sp)[i] = v;
-    reinterpret_cast<uint32_t*>(flag)[i] = 0u;
-    part += (static_cast<double>(v.x) + static_cast<double>(v.y)) +
-            (static_cast<double>(v.z) + static_cast<double>(v.w));
+  float pv[4 * G];
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    const int g = tid + k * kSipThreads;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (g < n_grp) v = __ldcs(pr + g);  // padding columns hold 0
+    pv[4 * k] = v.x;
+    pv[4 * k + 1] = v.y;
+    pv[4 * k + 2] = v.z;
+    pv[4 * k + 3] = v.w;
   }
-  double rest = block_sum_d(part, redd);  // its barriers also publish sp / flag
+  // elements past n_sub (padding) are 0 and are never capped or kept
+  uint32_t valid[MW];
+#pragma unroll
+  for (int w = 0; w < MW; ++w) valid[w] = 0u;
+#pragma unroll
+  for (int i = 0; i < 4 * G; ++i)
+    if (4 * (tid + (i >> 2) * kSipThreads) + (i & 3) < n_sub) valid[i >> 5] |= 1u << (i & 31);
+  // pairwise sum of the thread's uncapped p (capped elements masked out)
+  auto thread_sum = [&](const uint32_t (&capped)[MW]) -> double {
+    float t[4 * G];
+#pragma unroll
+    for (int i = 0; i < 4 * G; ++i) t[i] = (capped[i >> 5] >> (i & 31)) & 1u ? 0.f : pv[i];
+#pragma unroll
+    for (int w = 2 * G; w >= 1; w >>= 1)
+#pragma unroll
+      for (int i = 0; i < w; ++i) t[i] += t[i + w];
+    return static_cast<double>(t[0]);
+  };
+  uint32_t capped[MW];
+#pragma unroll
+  for (int w = 0; w < MW; ++w) capped[w] = ~valid[w];  // padding counts as capped, not in any sum
+  int slot = 0;
+  int dummy = 0;
+  double rest = thread_sum(capped);
+  block_sum2(dummy, rest, slot, rc, rd);
   // water filling
   int ncap = 0;
   double lam = 0.0;
   for (int round = 0; round <= n_sub && rest > 0.0; ++round) {
     lam = static_cast<double>(m - ncap) / rest;
+    const float lamf = static_cast<float>(lam);
     int newc = 0;
-    part = 0.0;
-    for (int j = tid; j < n_sub; j += kSipThreads) {
-      if (!flag[j]) {
-        const double pj = static_cast<double>(sp[j]);
-        if (lam * pj >= 1.0) {
-          flag[j] = 1;
-          ++newc;
-        } else {
-          part += pj;
-        }
+#pragma unroll
+    for (int i = 0; i < 4 * G; ++i) {
+      const uint32_t bit = 1u << (i & 31);
+      if (!(capped[i >> 5] & bit) && lamf * pv[i] >= 1.f) {
+        capped[i >> 5] |= bit;
+        ++newc;
       }
     }
-    int dummy;
-    const int tot = block_sum_i(newc, redi, dummy);
-    if (tot == 0) break;
-    ncap += tot;
-    rest = block_sum_d(part, redd);
+    double part = thread_sum(capped);
+    slot ^= 1;
+    block_sum2(newc, part, slot, rc, rd);
+    if (newc == 0) break;
+    ncap += newc;
+    rest = part;
   }
-  auto pi_of = [&](int j) -> double {
-    if (flag[j] & 1) return 1.0;
-    return fmin(1.0, lam * static_cast<double>(sp[j]));
+  const float lamf = static_cast<float>(lam);
+  // pi as fp32: 1 for capped, else min(1, lambda p)
+  auto pi_of = [&](int i) -> float {
+    if ((capped[i >> 5] >> (i & 31)) & 1u) return 1.f;
+    return fminf(1.f, lamf * pv[i]);
   };
   // draws
-  const int n_grp = ld / 4;
+  uint32_t kept[MW];
+#pragma unroll
+  for (int w = 0; w < MW; ++w) kept[w] = 0u;
   const uint32_t ctr = static_cast<uint32_t>(row);
-  auto mark = [&](int g, uint4 w) {
-    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int k = 0; k < G; k += 2) {
+    const int g0 = tid + k * kSipThreads, g1 = g0 + kSipThreads;
+    uint4 a = make_uint4(static_cast<uint32_t>(g0), 0u, ctr, 0u);
+    uint4 b = make_uint4(static_cast<uint32_t>(g1), 0u, ctr, 0u);
+    if (g0 < n_grp) philox4x32_10_x2(a, b, seed_lo, seed_hi);
+    const uint32_t xa[4] = {a.x, a.y, a.z, a.w}, xb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      const int j = 4 * g + e;
-      if (j < n_sub && static_cast<double>(x[e] >> 8) * (1.0 / 16777216.0) < pi_of(j))
-        flag[j] |= 2;
+      // u = (x >> 8) * 2^-24, exact in fp32
+      const int i0 = 4 * k + e, i1 = 4 * (k + 1) + e;
+      if (((valid[i0 >> 5] >> (i0 & 31)) & 1u) &&
+          static_cast<float>(xa[e] >> 8) * (1.f / 16777216.f) < pi_of(i0))
+        kept[i0 >> 5] |= 1u << (i0 & 31);
+      if (k + 1 < G && ((valid[i1 >> 5] >> (i1 & 31)) & 1u) &&
+          static_cast<float>(xb[e] >> 8) * (1.f / 16777216.f) < pi_of(i1))
+        kept[i1 >> 5] |= 1u << (i1 & 31);
     }
-  };
-  for (int g = tid; g < n_grp; g += 2 * kSipThreads) {
-    const int g2 = g + kSipThreads;
-    uint4 a = make_uint4(static_cast<uint32_t>(g), 0u, ctr, 0u);
-    uint4 b = make_uint4(static_cast<uint32_t>(g2), 0u, ctr, 0u);
-    philox4x32_10_x2(a, b, seed_lo, seed_hi);
-    mark(g, a);
-    if (g2 < n_grp) mark(g2, b);
+  }
+  // ascending output: exclusive scan of the kept counts of group k over the
+  // threads, offset by the totals of groups k' < k
+  int inc[G];
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    inc[k] = __popc((kept[(4 * k) >> 5] >> ((4 * k) & 31)) & 0xfu);
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, inc[k], o);
+      if (lane >= o) inc[k] += t;
+    }
+    if (lane == 31) tab[warp][k] = inc[k];
   }
   __syncthreads();
-  // ascending output
-  const int chunk = ((n_grp + kSipThreads - 1) / kSipThreads) * 4;
-  const int j_lo = min(ld, tid * chunk);
-  const int j_hi = min(ld, j_lo + chunk);
-  int mine = 0;
-  for (int j = j_lo; j < j_hi; j += 4)
-    mine += __popc(reinterpret_cast<const uint32_t*>(flag)[j >> 2] & 0x02020202u);
-  int before;
-  const int total = block_sum_i(mine, redi, before);
-  int pos = before;
+  int base = 0;
   int32_t* out = idx + static_cast<size_t>(row) * cap;
   float* lw = logw ? logw + static_cast<size_t>(row) * cap : nullptr;
-  for (int j = j_lo; j < j_hi; ++j) {
-    if (flag[j] & 2) {
-      if (pos < cap) {
-        out[pos] = j;
-        if (lw) lw[pos] = static_cast<float>(-log(pi_of(j)));
-      }
-      ++pos;
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kSipWarps; ++w) {
+      const int c = tab[w][k];
+      if (w < warp) before += c;
+      tot += c;
     }
+    const uint32_t bits = (kept[(4 * k) >> 5] >> ((4 * k) & 31)) & 0xfu;
+    int pos = base + before + inc[k] - __popc(bits);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (bits & (1u << e)) {
+        if (pos < cap) {
+          out[pos] = 4 * (tid + k * kSipThreads) + e;
+          if (lw) lw[pos] = -logf(pi_of(4 * k + e));
+        }
+        ++pos;
+      }
+    }
+    base += tot;
   }
   if (tid == 0) {
-    cnt[row] = min(total, cap);
-    if (required_cap) atomicMax(required_cap, total);
-    if (total > cap) raise_status(dev_status, STA_DEV_CAPACITY);
+    cnt[row] = min(base, cap);
+    if (required_cap) atomicMax(required_cap, base);
+    if (base > cap) raise_status(dev_status, STA_DEV_CAPACITY);
   }
 }
 
@@ -416,7 +458,9 @@ cudaError_t launch_kmeans_t(const __nv_bfloat16* q, float* cent, float* wts, int
 
 }  // namespace
 
-int ibcs_max_subblocks() { return static_cast<int>((200 * 1024) / (sizeof(float) + 1)); }
+// Sub-blocks per row the sampler holds in registers: 4 per group, up to 40
+// groups per thread.
+int ibcs_max_subblocks() { return 4 * 40 * kSipThreads; }
 
 cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
                           int d, int B, int km_k, int iters, cudaStream_t s) {
@@ -434,13 +478,20 @@ cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int h
 cudaError_t launch_sip_sample(const float* p, int rows, int n_sub, int m, uint64_t seed,
                               int32_t* idx, float* logw, int32_t* cnt, int cap,
                               int32_t* required_cap, int32_t* dev_status, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>((n_sub + 3) & ~3) * (sizeof(float) + 1);
-  cudaError_t e = set_dyn_smem<sip_sample_kernel>(static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  sip_sample_kernel<<<rows, kSipThreads, smem, s>>>(
-      p, n_sub, m, static_cast<uint32_t>(seed & 0xffffffffu), static_cast<uint32_t>(seed >> 32),
-      idx, logw, cnt, cap, required_cap, dev_status);
-  return cudaGetLastError();
+  const int n_grp = (n_sub + 3) / 4;
+  const uint32_t lo = static_cast<uint32_t>(seed & 0xffffffffu);
+  const uint32_t hi = static_cast<uint32_t>(seed >> 32);
+#define STA_SIP_CASE(GG)                                                                   \
+  if (n_grp <= GG * kSipThreads) {                                                         \
+    sip_sample_kernel<GG><<<rows, kSipThreads, 0, s>>>(p, n_sub, m, lo, hi, idx, logw, cnt, \
+                                                       cap, required_cap, dev_status);     \
+    return cudaGetLastError();                                                             \
+  }
+  STA_SIP_CASE(8)
+  STA_SIP_CASE(16)
+  STA_SIP_CASE(40)
+#undef STA_SIP_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace sta
