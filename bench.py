@@ -48,7 +48,7 @@ sys.path.insert(0, ROOT)
 METRIC = "effective TFLOP/s on retained blocks; speedup vs dense at same shape (1×B200)"
 DEFAULT_WORKLOAD = "ab_sampled"
 WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled", "tra_token",
-             "dynrad_static", "dynrad_dynamic")
+             "tra_token_tiled", "dynrad_static", "dynrad_dynamic")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 * 1024 * 1024
 
@@ -269,6 +269,13 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
         c = w["tra_token"]
         Hq = np.zeros(N)
         t_lists = 0.0
+        perm = None
+        if w.get("layout"):
+            # tile-major order: blocks are runs of positions of the permuted
+            # sequence; attention runs on the permuted rows
+            from oracle import tile_major
+            perm = tile_major.order(w["F"], w["H"], w["W"], *w["layout"])
+            qp, kp, vp = (tile_major.to_layout(x, perm) for x in (qh, kh, vh))
     elif sel == "dynrad":
         c = w["dynrad"]
         got = dynrad.select(qh, kh, w["F"], w["H"], w["W"], B, w["radial"], c["mode"],
@@ -285,13 +292,17 @@ def cpu_baseline(w, budget_s=15.0, seed=0):
             # the entropies are the warm-up's (not charged to the step); the
             # block lists and the attention are
             lo, hi = qb * B, min(N, qb * B + B)
-            Hq[lo:hi] = tra_token.query_entropy(qh[lo:hi], kh, 1.0 / np.sqrt(d))
+            toks = np.arange(lo, hi) if perm is None else perm[lo:hi]
+            Hq[toks] = tra_token.query_entropy(qh[toks], kh, 1.0 / np.sqrt(d))
             ts = time.perf_counter()
             ids, _ = tra_token.block_lists(Hq, w["F"], w["H"], w["W"], B, c["tau"], c["gamma"],
-                                           c["vote"], [qb])[qb]
+                                           c["vote"], [qb], perm=perm)[qb]
             t_lists += time.perf_counter() - ts
             ts = time.perf_counter()
-            block_sparse_rows(qh, kh, vh, qb, ids, B, U)
+            if perm is None:
+                block_sparse_rows(qh, kh, vh, qb, ids, B, U)
+            else:
+                block_sparse_rows(qp, kp, vp, qb, ids, B, U)
             t_att += time.perf_counter() - ts
             keys = sum(min(U, N - u * U) for u in ids)
             flops += 4.0 * d * (hi - lo) * keys
@@ -412,23 +423,45 @@ def main(argv=None):
     # token-level TRA: the per-query entropies come from a dense warm-up pass
     # (dense attention that also writes each query's entropy), run once and
     # reused by every step, as the pipeline reuses them across denoising steps
+    # tile-major token order (layout workloads): the attention runs on
+    # permuted copies of q, k, v and its output is permuted back; both
+    # permutations are part of the step
+    layout = w.get("layout")
+    if layout:
+        qt, kt, vt, ot = (torch.empty_like(qd) for _ in range(4))
+
+        def permute_in():
+            for x, y in ((qd, qt), (kd, kt), (vd, vt)):
+                sta.sta_permute_tokens(prob, layout[0], layout[1], 0, x, y)
+
+        def permute_out():
+            sta.sta_permute_tokens(prob, layout[0], layout[1], 1, ot, od)
+
+        permute_in()
+    else:
+        qt, kt, vt, ot = qd, kd, vd, od
     ent = None
     warm = None
-    if w["selector"] == "tra_token":
-        ent = torch.empty(w["heads"], w["N"], dtype=torch.float32, device="cuda")
+
+    def warmup_entropy(qq, kk, vv):
+        e = torch.empty(w["heads"], w["N"], dtype=torch.float32, device="cuda")
         ow = torch.empty_like(qd)
         stw = torch.zeros(1, dtype=torch.int32, device="cuda")
+        ms = None
         for i in range(4):
             a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a_.record()
-            sta.sta_dense_attn_entropy_fwd(session.problem(w), qd, kd, vd, 0.0, ow, ent,
+            sta.sta_dense_attn_entropy_fwd(session.problem(w), qq, kk, vv, 0.0, ow, e,
                                            dev_status=stw)
             b_.record()
             torch.cuda.synchronize()
-            warm = a_.elapsed_time(b_)
+            ms = a_.elapsed_time(b_)
         if int(stw.item()) != 0:
             raise RuntimeError("device status " + sta.sta_dev_status_string(int(stw.item())))
-        del ow
+        return e, ms
+
+    if w["selector"] == "tra_token":
+        ent, warm = warmup_entropy(qt, kt, vt)  # entropies by position of the sequence
     sel = session.selector(w, difd, entropy=ent)
     prm = session.attn_params(w)
     L = session.Lists(w)
@@ -439,15 +472,19 @@ def main(argv=None):
     l2_flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
 
     def select():
-        sta.sta_build_blocks(prob, sel, qd if needs_qk else None, kd if needs_qk else None,
+        sta.sta_build_blocks(prob, sel, qt if needs_qk else None, kt if needs_qk else None,
                              L.struct, workspace=sws, dev_status=st)
 
-    def attend(qq=qd, kk=kd, vv=vd, oo=od):
+    def attend(qq=qt, kk=kt, vv=vt, oo=ot):
         sta.sta_sparse_attn_fwd(prob, prm, qq, kk, vv, L.struct, oo, dev_status=st)
 
     def step():
+        if layout:
+            permute_in()
         select()
         attend()
+        if layout:
+            permute_out()
 
     for _ in range(args.warmup):
         step()
@@ -467,7 +504,10 @@ def main(argv=None):
     # the per-stage device times.
     graphs = {}
     try:
-        for name, fn in (("step", step), ("select", select), ("attend", attend)):
+        stages = [("step", step), ("select", select), ("attend", attend)]
+        if layout:
+            stages.append(("permute", lambda: (permute_in(), permute_out())))
+        for name, fn in stages:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 fn()
@@ -519,6 +559,30 @@ def main(argv=None):
     ms = max_over_ranks(sum(step_ms) / len(step_ms), ws)
     sel_avg = sum(sel_ms) / len(sel_ms)
     attn_avg = sum(attn_ms) / len(attn_ms)
+
+    layout_info = None
+    if layout:
+        run_perm = graphs["permute"].replay if graphs else (lambda: (permute_in(), permute_out()))
+        perm_ms = timed(run_perm, max(5, min(20, args.steps)))
+        perm_avg = sum(perm_ms) / len(perm_ms)
+        # q, k, v in and o out: each element read once and written once
+        pbytes = 4 * 2 * w["heads"] * w["N"] * w["d"] * 2
+        layout_info = {"tile": list(layout), "permute_ms": perm_avg, "permute_bytes": pbytes,
+                       "permute_gbs": pbytes / (perm_avg * 1e-3) / 1e9}
+        # the same pipeline in raster order on the same grid, for comparison
+        w_r = dict(w, layout=None)
+        ent_r, _ = warmup_entropy(qd, kd, vd)
+        sel_r = session.selector(w_r, None, entropy=ent_r)
+        L_r = session.Lists(w_r)
+        sta.sta_build_blocks(prob, sel_r, None, None, L_r.struct, dev_status=st)
+        torch.cuda.synchronize()
+        pairs_r = session.retained_pairs(w_r, L_r)
+        att_r = timed(lambda: sta.sta_sparse_attn_fwd(prob, prm, qd, kd, vd, L_r.struct, od,
+                                                      dev_status=st), max(5, min(20, args.steps)))
+        layout_info["raster_comparison"] = {
+            "retained_fraction": pairs_r / (w["N"] ** 2 * w["heads"]),
+            "attn_ms": sum(att_r) / len(att_r)}
+        del L_r, ent_r
 
     # dense at the same shape (the speedup denominator)
     def dense():
@@ -582,7 +646,8 @@ def main(argv=None):
                      "list_entries": entries},
         "e2e": {"value": total_flops / (e2e_avg * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_avg, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": (SELECTOR_LAUNCHES[w["selector"]] + 1) * args.steps,
+        "gpu_launches": (SELECTOR_LAUNCHES[w["selector"]] + 1 + (4 if layout else 0))
+                        * args.steps,
         "clocks": clk.summary(),
     }
     # Lists (and, for tra_token, entropies) reused across steps: a step is the
@@ -591,6 +656,10 @@ def main(argv=None):
                           "value": total_flops / (max_over_ranks(attn_avg, ws) * 1e-3) / 1e12,
                           "unit": "TFLOP/s",
                           "note": "selector run once, its lists reused by every step"}
+    if layout_info is not None:
+        hbm_pk = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        layout_info["permute_frac_of_hbm"] = layout_info["permute_gbs"] / hbm_pk
+        line["layout"] = layout_info
     if warm is not None:
         dflops = 4.0 * w["d"] * float(w["N"]) ** 2 * w["heads"]
         line["tra_warmup"] = {"ms": warm, "tflops": dflops / (warm * 1e-3) / 1e12,

@@ -120,6 +120,10 @@ typedef struct {
  *          (h_j - h_i)^2 + (w_j - w_i)^2 <= r_{f_j}^2.  A key block is listed
  *          for a query block iff at least tra_vote kept (query, key) pairs fall
  *          in the pair (token voting).  block_q == kv_unit; lists per head.
+ *          Blocks are runs of block_q sequence positions: raster order, or
+ *          with layout_tile_h, layout_tile_w > 0 the tile-major order of
+ *          sta_permute_tokens (2. Methodology, The TRA Pipeline, Efficient
+ *          Execution); tra_entropy is then indexed by tile-major position.
  * dynrad   [DYN] Abstract: the radial lists (radial_* parameters) are the
  *          candidates; p_c = softmax over the candidates of the pooled
  *          scores Qbar_b.Kbar_c/sqrt(d) (fp32); candidates ranked by score
@@ -153,6 +157,9 @@ typedef struct {
   /* dynrad (and the radial_* fields for its prior) */
   int dyn_mode;
   float dyn_ratio, dyn_threshold;
+  /* token order of the sequence the lists index (tra_token): 0, 0 = raster;
+   * tile_h x tile_w = tile-major (see sta_permute_tokens) */
+  int layout_tile_h, layout_tile_w;
 } sta_selector_params;
 
 /*
@@ -309,6 +316,27 @@ sta_status sta_sparse_attn_fwd_noalloc(const sta_problem* prob, const sta_attn_p
                                        const void* q, const void* k, const void* v,
                                        const sta_block_lists* lists, void* o,
                                        int32_t* dev_status, sta_stream_t stream);
+
+/*
+ * Token permutation between the raster order and a tile-major order
+ * ([TRA] 2. Methodology, The TRA Pipeline, Efficient Execution: tokens are
+ * reordered tile by tile so that a query's spatial neighbours are
+ * contiguous).  Within each frame, positions run over spatial tiles of
+ * tile_h x tile_w tokens: tile row, tile column, row inside the tile, column
+ * inside the tile.  Tiles on the bottom and right edges are cut by the grid
+ * (no padding), so the order is a permutation of the N tokens of each frame.
+ * tile_h = 1, tile_w = W is the raster order.
+ *   inverse = 0: out[h][j] = in[h][perm(j)]   (raster -> tile-major)
+ *   inverse = 1: out[h][perm(j)] = in[h][j]   (tile-major -> raster)
+ * with perm(j) the raster token at tile-major position j.  in, out: device
+ * tensors [heads][N][d] of prob->dtype, caller-owned, not overlapping.
+ * Attention in the tile-major order is the same attention: permute q, k, v,
+ * run the selector (layout_tile_h/w set) and sta_sparse_attn_fwd, and permute
+ * o back.  Errors: STA_ERR_ARG (null, overlap, tile_h or tile_w outside
+ * [1, H] x [1, W]), STA_ERR_CUDA.
+ */
+sta_status sta_permute_tokens(const sta_problem* prob, int tile_h, int tile_w, int inverse,
+                              const void* in, void* out, sta_stream_t stream);
 
 /* Static description of a status code / of the device status bits. */
 const char* sta_status_string(sta_status s);

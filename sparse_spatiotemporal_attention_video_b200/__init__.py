@@ -11,7 +11,7 @@ from ._lib import (AttnParams, BlockLists, Problem, SelectorParams, StaError, ST
                    STA_DEV_BAD_INDEX, STA_DEV_CAPACITY, STA_DEV_EMPTY_ROW, STA_DEV_TIMEOUT)
 from .api import (sta_attn_workspace, sta_build_blocks, sta_build_blocks_rows,
                   sta_build_blocks_workspace, sta_dense_attn_entropy_fwd, sta_dense_attn_fwd,
-                  sta_dev_status_string, sta_sparse_attn_fwd, sta_sparse_attn_fwd_noalloc,
-                  sta_status_string, sta_version)
+                  sta_dev_status_string, sta_permute_tokens, sta_sparse_attn_fwd,
+                  sta_sparse_attn_fwd_noalloc, sta_status_string, sta_version)
 
 _lib.load()

@@ -47,7 +47,8 @@ class SelectorParams(ctypes.Structure):
                 ("tra_tau", ctypes.c_float), ("tra_gamma", ctypes.c_float),
                 ("tra_vote", ctypes.c_int), ("tra_entropy", ctypes.c_void_p),
                 ("dyn_mode", ctypes.c_int), ("dyn_ratio", ctypes.c_float),
-                ("dyn_threshold", ctypes.c_float)]
+                ("dyn_threshold", ctypes.c_float),
+                ("layout_tile_h", ctypes.c_int), ("layout_tile_w", ctypes.c_int)]
 
 
 class BlockLists(ctypes.Structure):
@@ -95,6 +96,9 @@ SIGNATURES = {
                                                   ctypes.c_void_p, ctypes.c_void_p,
                                                   ctypes.c_size_t, ctypes.c_void_p,
                                                   ctypes.c_void_p]),
+    "sta_permute_tokens": (ctypes.c_int, [ctypes.POINTER(Problem), ctypes.c_int, ctypes.c_int,
+                                          ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p]),
     "sta_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sta_dev_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "sta_version": (ctypes.c_int, []),

@@ -105,6 +105,14 @@ def sta_dense_attn_entropy_fwd(prob, q, k, v, scale, o, entropy, workspace=None,
           "sta_dense_attn_entropy_fwd")
 
 
+def sta_permute_tokens(prob, tile_h, tile_w, inverse, x, out, stream=None):
+    """Raster <-> tile-major row permutation of a [heads][N][d] tensor (inverse=0:
+    raster to tile-major, 1: back)."""
+    lib = _lib.load()
+    check(lib.sta_permute_tokens(ctypes.byref(prob), int(tile_h), int(tile_w), int(inverse),
+                                 _ptr(x), _ptr(out), _stream(stream)), "sta_permute_tokens")
+
+
 def sta_status_string(code: int) -> str:
     return _lib.load().sta_status_string(code).decode()
 

@@ -24,6 +24,37 @@ __device__ __forceinline__ void raise_status(int32_t* dev_status, int32_t bits) 
   if (dev_status) atomicOr(dev_status, bits);
 }
 
+// Token layout of a sequence ("Token Radius Attention for Efficient Video
+// Generation", 2. Methodology, The TRA Pipeline, Efficient Execution: tokens
+// reordered tile by tile).  Within a frame, positions run over spatial tiles
+// of th x tw tokens: tile row, tile column, row in the tile, column in the
+// tile; tiles on the bottom and right edges are cut by the grid (no padding).
+// th = 1, tw = W is the raster order.
+struct TokLayout {
+  int H, W, th, tw;
+};
+
+// Grid coordinates (f, h, w) of the token at sequence position t, and the
+// number of positions from t on that continue along the same grid row (to
+// the end of the tile's row).
+__device__ __forceinline__ void layout_coords(const TokLayout& L, int t, int& f, int& h, int& w,
+                                              int& run) {
+  const int S = L.H * L.W;
+  f = t / S;
+  const int j = t - f * S;
+  const int tr = j / (L.th * L.W);       // tile row (every earlier one is full height)
+  const int rem = j - tr * L.th * L.W;
+  const int thr = min(L.th, L.H - tr * L.th);  // height of this tile row
+  const int tc = rem / (thr * L.tw);     // tile column (every earlier one is full width)
+  const int rem2 = rem - tc * thr * L.tw;
+  const int twc = min(L.tw, L.W - tc * L.tw);  // width of this tile
+  const int i = rem2 / twc;
+  const int c = rem2 - i * twc;
+  h = tr * L.th + i;
+  w = tc * L.tw + c;
+  run = twc - c;
+}
+
 enum AttnKind : int {
   kItemList = 0,       // raster query block, keys from a list row
   kItemDense = 1,      // raster query block, every key
@@ -72,6 +103,12 @@ cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tm_q,
                              int num_sms, cudaStream_t stream);
 cudaError_t launch_f32_to_bf16(const float* src, __nv_bfloat16* dst, size_t n, cudaStream_t s);
 
+// Row permutation between the raster and a tile-major layout (layout.cu):
+// out[h][j] = in[h][perm(j)] (inverse = 0) or out[h][perm(j)] = in[h][j]
+// (inverse = 1), rows of row_bytes (a multiple of 16).
+cudaError_t launch_permute_rows(const void* in, void* out, int heads, int N, int row_bytes,
+                                const TokLayout& L, int inverse, cudaStream_t s);
+
 // Radial selector (sel_radial.cu).
 cudaError_t launch_radial_lists(int F, int H, int W, int B, int w0, int w_off, int full_df,
                                 int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
@@ -115,9 +152,9 @@ cudaError_t launch_entropy_lists(const float* qbar, const float* kbar, float* sc
 int tra_max_frames();
 int tra_max_block();
 cudaError_t launch_tra_token_lists(const float* entropy, int heads, int F, int H, int W, int B,
-                                   float tau, float gamma, int vote, int32_t* idx, int32_t* cnt,
-                                   int cap, int32_t* required_cap, int32_t* dev_status,
-                                   cudaStream_t s);
+                                   int tile_h, int tile_w, float tau, float gamma, int vote,
+                                   int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
+                                   int32_t* dev_status, cudaStream_t s);
 
 // Dual-mode selection in the radial prior (sel_dynrad.cu).
 int dynrad_max_candidates();

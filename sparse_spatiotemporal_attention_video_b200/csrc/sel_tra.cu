@@ -16,18 +16,27 @@
 //   key block kb listed for query block qb iff at least `vote` kept pairs
 //   (i in qb, j in kb).
 //
-// One CTA per (query block, head).  The block's queries (coordinates and
-// r0^2) and the per-distance decay table are staged in shared memory; thread
-// t then takes key blocks t, t + 256, ...: it splits the block's tokens into
-// grid-row segments [w0, w1] of one (f, h) and, per query, counts the keys
+// Blocks are runs of B consecutive sequence positions, in the raster order or
+// in a tile-major order (tokens reordered tile by tile, The TRA Pipeline,
+// Efficient Execution); a position's grid coordinates come from
+// layout_coords.  One CTA per (query block, head).  The block's queries
+// (coordinates and r0^2) and the per-distance decay table are staged in
+// shared memory; thread t then takes key blocks t, t + 256, ...: it splits
+// the block's positions into grid-row segments [w0, w1] of one (f, h) (in a
+// tile-major order a segment ends at the tile's edge) and, per query, counts
+// the keys
 // of each segment inside the query's disk: with rest = r_f^2 - dh^2 >= 0
 // (exact in fp32: dh^2 is an integer below 2^24) and dw = floor(sqrt(rest))
 // (corrected so that dw^2 <= rest < (dw+1)^2 exactly), the row's kept
 // columns are [w_i - dw, w_i + dw].  A segment is skipped without visiting
 // the queries when no query can reach it: per frame, the largest r_f^2 over
 // the block's queries (frames whose share is below one token excluded)
-// against the squared row distance from the block's row span.  Kept blocks
-// are compacted in ascending order with warp ballots and a block-wide scan.
+// against the squared row distance from the block's row span.  With vote 1
+// (any kept pair lists the block) the segments are merged into maximal
+// rectangles and each (rectangle, query) pair takes one test of its nearest
+// key: for a 16 x 8 tile block that is one test per query instead of 16.
+// Kept blocks are compacted in ascending order with warp ballots and a
+// block-wide scan.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -41,8 +50,9 @@ constexpr int kTraMaxQ = 128;   // query block size limit
 constexpr int kTraMaxF = 1024;  // frame count limit (decay table)
 
 struct TraArgs {
-  const float* entropy;  // [heads][N]
+  const float* entropy;  // [heads][N], indexed by sequence position
   int heads, F, H, W, B, nb;
+  TokLayout L;           // token order of the sequence (raster or tile-major)
   float tau, gamma;
   int vote;
   int32_t* idx;
@@ -83,11 +93,12 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
   __syncthreads();
   const float* Hh = a.entropy + static_cast<size_t>(head) * N;
   for (int r = threadIdx.x; r < nq; r += kTraThreads) {
-    const int t = q0 + r;
-    const int f = t / S, rem = t - f * S;
+    const int t = q0 + r;  // sequence position
+    int f, h, w, run;
+    layout_coords(a.L, t, f, h, w, run);
     qf[r] = f;
-    qh[r] = rem / a.W;
-    qw[r] = rem - qh[r] * a.W;
+    qh[r] = h;
+    qw[r] = w;
     float G = 0.f;  // frames in order: the same sum on every query of frame f
     for (int f2 = 0; f2 < a.F; ++f2) G += decay[abs(f2 - f)];
     const float n = a.tau * expf(__ldg(Hh + t));
@@ -111,16 +122,57 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
   for (int c0 = 0; c0 < a.nb; c0 += kTraThreads) {
     const int kb = c0 + threadIdx.x;
     bool keep = false;
-    if (kb < a.nb) {
+    if (kb < a.nb && a.vote == 1) {
+      // vote 1: the block is kept iff one of its maximal key rectangles
+      // (grid-row segments of one frame, vertically merged when consecutive
+      // rows span the same columns) has its key nearest to some query inside
+      // that query's disk; the nearest key minimises the squared distance
+      // over the rectangle, so one integer test per (rectangle, query)
+      // decides it
+      const int t0 = kb * a.B, t1 = min(N, t0 + a.B);
+      auto test_rect = [&](int f, int h0, int h1, int w0, int w1) -> bool {
+        const int drow = max(0, max(h0 - hmax, hmin - h1));
+        if (static_cast<float>(drow * drow) > reach[f]) return false;  // no query reaches it
+        for (int r = 0; r < nq; ++r) {
+          const float rf = qr0[r] * decay[abs(f - qf[r])];
+          if (rf * 3.14159265358979f < 1.f) continue;  // share below one token
+          const int dh = max(0, max(h0 - qh[r], qh[r] - h1));
+          const int dw = max(0, max(w0 - qw[r], qw[r] - w1));
+          if (static_cast<float>(dh * dh + dw * dw) <= rf) return true;  // exact integers
+        }
+        return false;
+      };
+      bool have = false;
+      int cf = 0, ch0 = 0, ch1 = 0, cw0 = 0, cw1 = 0;  // rectangle being grown
+      for (int t = t0; t < t1 && !keep;) {
+        int f, h, w0, run;
+        layout_coords(a.L, t, f, h, w0, run);
+        const int len = min(run, t1 - t);
+        const int w1 = w0 + len - 1;
+        t += len;
+        if (have && f == cf && h == ch1 + 1 && w0 == cw0 && w1 == cw1) {
+          ch1 = h;
+          continue;
+        }
+        if (have) keep = test_rect(cf, ch0, ch1, cw0, cw1);
+        have = true;
+        cf = f;
+        ch0 = ch1 = h;
+        cw0 = w0;
+        cw1 = w1;
+      }
+      if (!keep && have) keep = test_rect(cf, ch0, ch1, cw0, cw1);
+    } else if (kb < a.nb) {
       const int t0 = kb * a.B, t1 = min(N, t0 + a.B);  // [t0, t1)
       const float wsq = static_cast<float>(a.W) * static_cast<float>(a.W);
       int votes = 0;
       // grid-row segments [w0, w1] of one (f, h) of the key block
       for (int t = t0; t < t1 && votes < a.vote;) {
-        const int f = t / S, rem = t - f * S;
-        const int h = rem / a.W, w0 = rem - h * a.W;
-        const int w1 = min(a.W - 1, w0 + (t1 - 1 - t));  // inclusive
-        t += w1 - w0 + 1;
+        int f, h, w0, run;
+        layout_coords(a.L, t, f, h, w0, run);
+        const int len = min(run, t1 - t);
+        const int w1 = w0 + len - 1;  // inclusive
+        t += len;
         const int drow = max(0, max(hmin - h, h - hmax));
         if (static_cast<float>(drow * drow) > reach[f]) continue;  // no query reaches it
         for (int r = 0; r < nq && votes < a.vote; ++r) {
@@ -163,15 +215,16 @@ int tra_max_frames() { return kTraMaxF; }
 int tra_max_block() { return kTraMaxQ; }
 
 cudaError_t launch_tra_token_lists(const float* entropy, int heads, int F, int H, int W, int B,
-                                   float tau, float gamma, int vote, int32_t* idx, int32_t* cnt,
-                                   int cap, int32_t* required_cap, int32_t* dev_status,
-                                   cudaStream_t s) {
+                                   int tile_h, int tile_w, float tau, float gamma, int vote,
+                                   int32_t* idx, int32_t* cnt, int cap, int32_t* required_cap,
+                                   int32_t* dev_status, cudaStream_t s) {
   TraArgs a;
   a.entropy = entropy;
   a.heads = heads;
   a.F = F;
   a.H = H;
   a.W = W;
+  a.L = TokLayout{H, W, tile_h, tile_w};
   a.B = B;
   const long long N = static_cast<long long>(F) * H * W;
   a.nb = static_cast<int>((N + B - 1) / B);

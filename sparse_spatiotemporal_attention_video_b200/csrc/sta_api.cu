@@ -15,7 +15,7 @@ using namespace sta;
 
 namespace {
 
-constexpr int kVersion = 100;  // 0.1.0
+constexpr int kVersion = 200;  // 0.2.0 (selector parameters gained the token layout)
 
 // Last CUDA error a call of this thread ran into (sta_last_cuda_error).
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
@@ -386,8 +386,12 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
           prob->F > tra_max_frames())
         return STA_ERR_UNSUPPORTED;
       out->head_shared = 0;
+      const int th = sel->layout_tile_h, tw = sel->layout_tile_w;
+      if ((th == 0) != (tw == 0) || th < 0 || tw < 0 || th > prob->H || tw > prob->W)
+        return STA_ERR_ARG;
       if (failed(launch_tra_token_lists(sel->tra_entropy, prob->heads, prob->F, prob->H, prob->W,
-                                        sel->block_q, sel->tra_tau, sel->tra_gamma,
+                                        sel->block_q, th == 0 ? 1 : th, th == 0 ? prob->W : tw,
+                                        sel->tra_tau, sel->tra_gamma,
                                         sel->tra_vote, out->idx, out->cnt, out->cap,
                                         out->required_cap, dev_status, s)))
         return STA_ERR_CUDA;
@@ -599,6 +603,25 @@ sta_status sta_dense_attn_entropy_fwd(const sta_problem* prob, const void* q, co
   if (!entropy) return STA_ERR_ARG;
   return dense_attn(prob, q, k, v, scale, o, entropy, workspace, workspace_bytes, dev_status,
                     stream);
+}
+
+sta_status sta_permute_tokens(const sta_problem* prob, int tile_h, int tile_w, int inverse,
+                              const void* in, void* out, sta_stream_t stream) {
+  sta_status st = check_problem(prob);
+  if (st != STA_OK) return st;
+  if (!in || !out || tile_h < 1 || tile_w < 1 || tile_h > prob->H || tile_w > prob->W)
+    return STA_ERR_ARG;
+  const int N = prob->F * prob->H * prob->W;
+  const size_t elem = prob->dtype == STA_F32 ? 4 : 2;
+  const size_t bytes = static_cast<size_t>(prob->heads) * N * prob->d * elem;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(in), b = reinterpret_cast<uintptr_t>(out);
+  if (a < b + bytes && b < a + bytes) return STA_ERR_ARG;  // overlapping buffers
+  if (a % 16 != 0 || b % 16 != 0) return STA_ERR_ARG;
+  const TokLayout L{prob->H, prob->W, tile_h, tile_w};
+  if (failed(launch_permute_rows(in, out, prob->heads, N, static_cast<int>(prob->d * elem), L,
+                                 inverse ? 1 : 0, reinterpret_cast<cudaStream_t>(stream))))
+    return STA_ERR_CUDA;
+  return STA_OK;
 }
 
 }  // extern "C"

@@ -48,6 +48,8 @@ def selector(w, difficulty=None, entropy=None):
     elif w["selector"] == "tra_token":
         c = w["tra_token"]
         s.tra_tau, s.tra_gamma, s.tra_vote = c["tau"], c["gamma"], c["vote"]
+        if w.get("layout"):
+            s.layout_tile_h, s.layout_tile_w = w["layout"]
         if entropy is not None:
             s.tra_entropy = api._ptr(entropy)
     return s

@@ -110,6 +110,11 @@ def test_next_selector_argument_checks(lib):
     assert build(tra, Problem(1, 2000, 4, 4, 64, 0)) == STA_ERR_UNSUPPORTED  # > frame limit
     assert lib.sta_build_blocks_rows(ctypes.byref(good), ctypes.byref(tra)) == 2 * 2
     assert lib.sta_build_blocks_workspace(ctypes.byref(good), ctypes.byref(tra)) == 0
+    # tile-major token order: both tile sides or neither, within the grid
+    for th, tw in ((4, 0), (0, 4), (-1, 4), (9, 4), (4, 9)):
+        tra.layout_tile_h, tra.layout_tile_w = th, tw
+        assert build(tra) == STA_ERR_ARG, (th, tw)
+    tra.layout_tile_h = tra.layout_tile_w = 0
 
     dyn = SelectorParams()
     dyn.kind, dyn.block_q, dyn.kv_unit = STA_SEL_DYNRAD, 128, 128
@@ -160,3 +165,23 @@ def test_package_exports_every_selector_kind(lib):
     assert len(kinds) == 6
     for n in kinds:
         assert getattr(pkg, n) == getattr(_lib, n), n
+
+
+def test_permute_tokens_argument_checks(lib):
+    """sta_permute_tokens rejects null and overlapping buffers and tiles
+    outside the grid before any launch."""
+    from sparse_spatiotemporal_attention_video_b200._lib import (STA_ERR_ARG,
+                                                                 STA_ERR_UNSUPPORTED, Problem)
+    good = Problem(2, 4, 8, 8, 64, 0)        # bf16 rows of 128 bytes, 2 x 256 rows: 64 KiB
+    a, b = ctypes.c_void_p(1 << 20), ctypes.c_void_p(1 << 24)
+
+    def perm(th, tw, x=a, y=b, prob=good):
+        return lib.sta_permute_tokens(ctypes.byref(prob), th, tw, 0, x, y, None)
+
+    assert perm(4, 4, None, b) == STA_ERR_ARG
+    assert perm(4, 4, a, None) == STA_ERR_ARG
+    for th, tw in ((0, 4), (4, 0), (9, 4), (4, 9), (-2, 2)):
+        assert perm(th, tw) == STA_ERR_ARG, (th, tw)
+    assert perm(4, 4, a, ctypes.c_void_p((1 << 20) + 4096)) == STA_ERR_ARG  # overlap
+    assert perm(4, 4, a, ctypes.c_void_p((1 << 24) + 8)) == STA_ERR_ARG    # not 16-byte aligned
+    assert perm(4, 4, prob=Problem(2, 4, 8, 8, 96, 0)) == STA_ERR_UNSUPPORTED

@@ -7,7 +7,7 @@ import math
 import numpy as np
 import pytest
 
-from oracle import tra_token
+from oracle import tile_major, tra_token
 
 
 def test_entropy_of_equal_logits_is_ln_n():
@@ -193,6 +193,65 @@ def test_vote_one_equals_nearest_key_of_each_row_segment(F, Hh, W, B, seed, tau)
         sizes.append(len(ids))
     nb = (N + B - 1) // B
     assert 0 < min(sizes) and max(sizes) < nb  # neither empty nor dense rows
+
+
+def _rectangles(block_tokens, S, W):
+    """Maximal key rectangles of one block: the block's tokens (raster ids,
+    in sequence order) cut into runs along grid rows, and runs of
+    consecutive rows with the same column range merged (f, h0, h1, w0, w1)."""
+    runs = []
+    for t in block_tokens:
+        f, h, w = t // S, (t % S) // W, t % W
+        if runs and runs[-1][:2] == [f, h] and runs[-1][3] == w - 1:
+            runs[-1][3] = w
+        else:
+            runs.append([f, h, w, w])
+    rects = []
+    for f, h, w0, w1 in runs:
+        if rects and rects[-1][0] == f and rects[-1][2] == h - 1 and rects[-1][3:] == [w0, w1]:
+            rects[-1][2] = h
+        else:
+            rects.append([f, h, h, w0, w1])
+    return rects
+
+
+@pytest.mark.parametrize("F,Hh,W,th,tw,B,seed", [(2, 12, 16, 4, 8, 32, 0), (3, 10, 13, 4, 4, 16, 1),
+                                                 (2, 9, 20, 3, 20, 24, 2), (2, 8, 8, 1, 8, 16, 3)])
+def test_vote_one_equals_nearest_key_of_each_rectangle(F, Hh, W, th, tw, B, seed):
+    """With vote 1 a key block is listed iff, for some query of the block, the
+    key of one of the block's maximal rectangles nearest to the query
+    (row clamp(h_i, h0, h1), column clamp(w_i, w0, w1)) is kept: inside a
+    rectangle of one frame that key minimises the squared distance, and the
+    frame's share does not depend on the key.  Tile-major orders with ragged
+    tiles, blocks that cut tiles, and the raster order (t_h = 1, t_w = W)."""
+    N, S = F * Hh * W, Hh * W
+    perm = tile_major.order(F, Hh, W, th, tw)
+    H = np.random.default_rng(seed).uniform(1.0, 4.0, N)
+    tau, gamma = 0.12, 0.3
+    got = tra_token.block_lists(H, F, Hh, W, B, tau, gamma, vote=1, perm=perm)
+    nb = (N + B - 1) // B
+    rects = [_rectangles(perm[kb * B:min(N, kb * B + B)], S, W) for kb in range(nb)]
+    sizes = []
+    for qb in range(nb):
+        kept = set()
+        for i in perm[qb * B:min(N, qb * B + B)]:
+            fi, hi, wi = i // S, (i % S) // W, i % W
+            r2 = tra_token.radius2(H[i], fi, F, tau, gamma)
+            for kb in range(nb):
+                if kb in kept:
+                    continue
+                for f, h0, h1, w0, w1 in rects[kb]:
+                    if np.pi * r2[f] < 1.0:
+                        continue
+                    hn, wn = min(max(hi, h0), h1), min(max(wi, w0), w1)
+                    if (hn - hi) ** 2 + (wn - wi) ** 2 <= r2[f]:
+                        kept.add(kb)
+                        break
+        ids, amb = got[qb]
+        assert len(amb) == 0
+        assert ids.tolist() == sorted(kept), qb
+        sizes.append(len(ids))
+    assert 0 < min(sizes) and max(sizes) < nb
 
 
 @pytest.mark.parametrize("delta,near", [(1e-5, True), (-1e-5, True), (4e-5, False),
