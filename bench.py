@@ -52,10 +52,13 @@ WORKLOADS = ("wan_radial", "tra_entropy", "heta_routed", "ab_sampled", "tra_toke
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 * 1024 * 1024
 
-# DRAM traffic of one attention launch from an ncu capture, valid only for
-# the kernel source it was taken on (sha256 of attn_fwd.cu, first 16 hex).
-NCU_TRAFFIC = {"source_sha": "8c8e5398b9d4d3c5", "workload": "wan_radial",
-               "bytes_per_launch": 302877440 + 84381696}
+# DRAM traffic of one attention launch (dram__bytes_read.sum +
+# dram__bytes_write.sum) from an ncu capture, valid only for the kernel
+# source it was taken on (sha256 of attn_fwd.cu, first 16 hex).  Captured on
+# 2 of the 24 heads (one launch, inputs larger than L2) and scaled by 12:
+# every head carries the same work.
+NCU_TRAFFIC = {"ab_sampled": {"source_sha": "9af626cd5e3bea6c",
+                              "bytes_per_launch": 12 * (439706880 + 70045184)}}
 
 
 def parse(argv=None):
@@ -620,8 +623,9 @@ def main(argv=None):
     hbm = float(pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     achieved = flops / (attn_avg * 1e-3) / 1e12
     traffic = None
-    if NCU_TRAFFIC["source_sha"] == source_sha() and NCU_TRAFFIC["workload"] == w["name"]:
-        traffic = NCU_TRAFFIC["bytes_per_launch"]
+    rec = NCU_TRAFFIC.get(w["name"])
+    if rec and rec["source_sha"] == source_sha() and not args.heads:
+        traffic = rec["bytes_per_launch"]
     sbytes, sbound = selector_bytes(w, entries)
     sel_gbs = sbytes / (sel_avg * 1e-3) / 1e9
     total_flops = sum_over_ranks(flops, ws)

@@ -929,16 +929,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool il = kInterleaved && !dense_like;
       const int nops = il ? I.upt : I.upt * L::DH;
       const int n_il = (a.N & ~7) / UNIT;  // units the interleaved view covers
+      const int n_units = (a.N + unit - 1) / unit;
+      // one lane per (slot, half) copy, or per slot in the interleaved layout
+      const int s = il ? lane : lane / L::DH, h = il ? 0 : lane % L::DH;
+      // List entries are fetched one tile ahead, so that their load latency
+      // is not on the path from a free ring slot to the copies into it.
+      auto fetch = [&](int t, int& e, bool& present) {
+        present = false;
+        e = 0;
+        if (!dense_like && lane < nops && t < I.ntiles) {
+          const int pos = t * I.upt + s;
+          if (pos < I.cnt) {
+            present = true;
+            e = __ldg(a.idx + static_cast<size_t>(I.row) * a.cap + pos);
+          }
+        }
+      };
+      int e_next;
+      bool p_next;
+      fetch(0, e_next, p_next);
       for (int t = 0; t < I.ntiles; ++t) {
-        // one lane per (slot, half) copy, or per slot in the interleaved layout
         int u = 0;
-        const int s = il ? lane : lane / L::DH, h = il ? 0 : lane % L::DH;
         if (lane < nops) {
-          int nv;
-          float lw;
-          bool bad;
-          u = slot_unit(a, I, t, s, nv, lw, bad);
-          if (bad && !is_v) raise_status(a.dev_status, STA_DEV_BAD_INDEX);
+          if (dense_like) {
+            u = t;
+          } else {
+            const int e = e_next;
+            const bool present = p_next;
+            fetch(t + 1, e_next, p_next);
+            // an out-of-range entry loads unit 0 (the softmax masks its slot)
+            const bool valid = present && e >= 0 && e < n_units;
+            if (present && !valid && !is_v) raise_status(a.dev_status, STA_DEV_BAD_INDEX);
+            u = valid ? e : 0;
+          }
         }
         const uint32_t st = n % RS;
         if (lane == 0) ok = mbar_wait(ring_empty + st, ((n / RS) & 1) ^ 1, abort, limit);
