@@ -35,8 +35,9 @@
 // (any kept pair lists the block) the segments are merged into maximal
 // rectangles and each (rectangle, query) pair takes one test of its nearest
 // key: for a 16 x 8 tile block that is one test per query instead of 16.
-// Kept blocks are compacted in ascending order with warp ballots and a
-// block-wide scan.
+// Key blocks are decided into a shared bitmask (no barriers between a
+// thread's blocks, whose costs differ widely) and compacted in ascending
+// order with one block-wide scan per 8,192 blocks.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -48,6 +49,7 @@ namespace {
 constexpr int kTraThreads = 256;
 constexpr int kTraMaxQ = 128;   // query block size limit
 constexpr int kTraMaxF = 1024;  // frame count limit (decay table)
+constexpr int kTraChunk = 32 * kTraThreads;  // key blocks decided per compaction
 
 struct TraArgs {
   const float* entropy;  // [heads][N], indexed by sequence position
@@ -77,6 +79,7 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
   __shared__ int qf[kTraMaxQ], qh[kTraMaxQ], qw[kTraMaxQ];
   __shared__ float reach[kTraMaxF];   // per frame: max r_f^2 over the block's queries
   __shared__ int warp_tot[kTraThreads / 32];
+  __shared__ uint32_t keepbits[kTraChunk / 32];  // decided key blocks of a chunk
   __shared__ int running, hmin, hmax;
   const int qb = blockIdx.x, head = blockIdx.y;
   const int S = a.H * a.W;
@@ -119,10 +122,11 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(head) * a.nb + qb;
   int32_t* out = a.idx + row * a.cap;
-  for (int c0 = 0; c0 < a.nb; c0 += kTraThreads) {
-    const int kb = c0 + threadIdx.x;
+  // Is key block kb listed?  (No barriers inside: threads take their key
+  // blocks at their own pace.)
+  auto decide = [&](int kb) -> bool {
     bool keep = false;
-    if (kb < a.nb && a.vote == 1) {
+    if (a.vote == 1) {
       // vote 1: the block is kept iff one of its maximal key rectangles
       // (grid-row segments of one frame, vertically merged when consecutive
       // rows span the same columns) has its key nearest to some query inside
@@ -162,7 +166,7 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
         cw1 = w1;
       }
       if (!keep && have) keep = test_rect(cf, ch0, ch1, cw0, cw1);
-    } else if (kb < a.nb) {
+    } else {
       const int t0 = kb * a.B, t1 = min(N, t0 + a.B);  // [t0, t1)
       const float wsq = static_cast<float>(a.W) * static_cast<float>(a.W);
       int votes = 0;
@@ -189,16 +193,40 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
       }
       keep = votes >= a.vote;
     }
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) warp_tot[warp] = __popc(bal);
+    return keep;
+  };
+  // Key blocks are decided kTraChunk at a time into a bitmask, then
+  // compacted in ascending order: thread t takes word t of the mask, an
+  // exclusive block scan of the words' bit counts places their ids.
+  for (int c0 = 0; c0 < a.nb; c0 += kTraChunk) {
+    const int c1 = min(a.nb, c0 + kTraChunk);
+    for (int wd = threadIdx.x; wd < kTraChunk / 32; wd += kTraThreads) keepbits[wd] = 0u;
+    __syncthreads();
+    for (int kb = c0 + threadIdx.x; kb < c1; kb += kTraThreads)
+      if (decide(kb)) atomicOr(&keepbits[(kb - c0) >> 5], 1u << ((kb - c0) & 31));
+    __syncthreads();
+    const int nwords = (c1 - c0 + 31) >> 5;  // <= kTraChunk / 32 <= kTraThreads
+    const uint32_t bits = threadIdx.x < nwords ? keepbits[threadIdx.x] : 0u;
+    const int cntw = __popc(bits);
+    int inc = cntw;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += t;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
     __syncthreads();
     int before = running;
-    for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    const int pos = before + __popc(bal & ((1u << lane) - 1u));
-    if (keep && pos < a.cap) out[pos] = kb;
+    for (int wd = 0; wd < warp; ++wd) before += warp_tot[wd];
+    int pos = before + inc - cntw;
+    for (uint32_t b = bits; b; b &= b - 1u) {
+      const int kb = c0 + threadIdx.x * 32 + (__ffs(b) - 1);
+      if (pos < a.cap) out[pos] = kb;
+      ++pos;
+    }
     __syncthreads();
     if (threadIdx.x == 0)
-      for (int w = 0; w < kTraThreads / 32; ++w) running += warp_tot[w];
+      for (int wd = 0; wd < kTraThreads / 32; ++wd) running += warp_tot[wd];
     __syncthreads();
   }
   if (threadIdx.x == 0) {
