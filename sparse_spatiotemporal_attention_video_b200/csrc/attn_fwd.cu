@@ -457,6 +457,10 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
   const float inv_scale = kLog2e / scale_log2;  // natural-log weight -> raw logit units
   const uint64_t limit = kWaitLimitNs;
   volatile int* abort = sh.abort;
+  // (m, l) of each row exchanged by the two groups at the end of an item
+  // (with the entropy terms z, a): [group][row]
+  __shared__ __align__(16) float4 xch4[ENT ? 256 : 1];
+  __shared__ __align__(16) float2 xch2[ENT ? 1 : 256];
   uint32_t g = 0, nitem = 0;
   bool ok = true;
   for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
@@ -649,31 +653,31 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
     if (!ok) break;
     // ------------------------------------------------------------ epilogue
     const uint32_t gl = g + I.ntiles - 1;  // last tile of the item
-    // The two groups exchange (m, l) of each row through TMEM: group J
-    // writes its pair into columns 64J+32, 64J+33 of the last tile's S
-    // buffer (its own half, which only it reads and has already read; the
-    // tile's P, which its PV still reads, is in columns 64J..64J+31), at the
-    // row's lane.  The MMA issuer writes the buffer again (the QK of tile
-    // gl+2) only after both groups have finished this epilogue (o_free).
-    const uint32_t tX = tmem + lane_off + (gl & 1) * 128 + 32;
-    tmem_st2(tX + 64 * J, __float_as_uint(m_run), __float_as_uint(l_run));
-    if constexpr (ENT) tmem_st2(tX + 64 * J + 2, __float_as_uint(z_run), __float_as_uint(a_run));
-    tmem_wait_st();
-    tc_fence_before();
+    // The two groups exchange (m, l) of each row through shared memory, so
+    // that no S buffer is held by the epilogue and the next item's QK
+    // products need not wait for it.  A group rewrites its slot only at the
+    // end of its next item, after the other group has read this one (it
+    // took part in every tile of that item).
+    if constexpr (ENT)
+      xch4[J * 128 + r] = make_float4(m_run, l_run, z_run, a_run);
+    else
+      xch2[J * 128 + r] = make_float2(m_run, l_run);
     __syncwarp();
     if (lane == 0) mbar_arrive(sh.lbar + quad);
     bool okw = __all_sync(0xffffffffu, mbar_wait(sh.lbar + quad, nitem & 1, abort, limit));
     float mo = 0.f, lo = 0.f, zo = 0.f, ao = 0.f;
     if (okw) {
-      tc_fence_after();
-      uint32_t um, ul, uz = 0, ua = 0;
-      tmem_ld2(tX + 64 * (1 - J), um, ul);
-      if constexpr (ENT) tmem_ld2(tX + 64 * (1 - J) + 2, uz, ua);
-      tmem_wait_ld();
-      mo = __uint_as_float(um);
-      lo = __uint_as_float(ul);
-      zo = __uint_as_float(uz);
-      ao = __uint_as_float(ua);
+      if constexpr (ENT) {
+        const float4 xo = xch4[(1 - J) * 128 + r];
+        mo = xo.x;
+        lo = xo.y;
+        zo = xo.z;
+        ao = xo.w;
+      } else {
+        const float2 xo = xch2[(1 - J) * 128 + r];
+        mo = xo.x;
+        lo = xo.y;
+      }
     }
     // the commit after the item's last PV covers every earlier MMA
     if (okw)
@@ -998,13 +1002,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t kt = 0, vt = 0, qn = 0, g = 0;
       bool ok = true;
       // first: the next PV starts the accumulators O_0 / O_1 of this item.
-      // O_0/O_1 and the (m, l) exchange columns of an item's last S buffer
-      // stay in use until both softmax groups have finished the item's
-      // epilogue (o_free, one phase per item): nfree counts the phases seen.
-      // The first PV of item qn, and the QK into the last S buffer of item
-      // qn-1 (tile xtile = its last tile + 2), wait for epilogues 0..qn-1.
+      // O_0/O_1 stay in use until both softmax groups have finished the
+      // item's epilogue (o_free, one phase per item): nfree counts the
+      // phases seen.  The first PV of item qn waits for epilogues 0..qn-1.
       bool first = true;
-      uint32_t nfree = 0, xtile = 0xffffffffu;
+      uint32_t nfree = 0;
       auto ensure_free = [&](uint32_t k) -> bool {
         while (nfree < k) {
           if (!mbar_wait(o_free, nfree & 1, abort, limit)) return false;
@@ -1059,10 +1061,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          if (g + t == xtile && !ensure_free(qn)) {
-            ok = false;
-            break;
-          }
           tc_fence_after();
           const uint32_t sb = (g + t) & 1;
           const uint32_t tS = tmem + sb * 128;
@@ -1091,7 +1089,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ++qn;
         g += I.ntiles;
-        xtile = g + 1;
       }
       if (!ok) fail(abort, a.dev_status);
       // all issued MMAs complete before TMEM is released
