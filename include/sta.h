@@ -27,6 +27,9 @@
  *   In-kernel errors are OR-ed into the caller's device word `dev_status`
  *   (an int32 in device memory, may be NULL) as STA_DEV_* bits; decode it
  *   after synchronising with sta_dev_status_string().
+ * - Each call that enqueues selector, attention or permutation work is
+ *   wrapped in an NVTX range named after the call (seen by profilers that
+ *   trace NVTX; free otherwise).
  * - Shapes supported: d in {64, 128}; block_q in {16, 32, 64, 128};
  *   kv_unit in {16, 32, 64, 128}.  Anything else returns STA_ERR_UNSUPPORTED.
  *   There is no CPU path.
@@ -69,6 +72,8 @@ typedef enum {
 #define STA_DEV_EMPTY_ROW 0x4  /* a query row had no kept key; its output is 0      */
 #define STA_DEV_BAD_INDEX 0x8  /* a list entry was out of range and was skipped     */
 #define STA_DEV_RANGE     0x10 /* an importance operand exceeded the fp16 range     */
+#define STA_DEV_DEBUG     0x20 /* debug build only: an index check failed and the
+                                  access it guarded was skipped                    */
 
 typedef enum { STA_BF16 = 0, STA_F32 = 1 } sta_dtype;
 
@@ -361,6 +366,28 @@ const char* sta_last_cuda_error(void);
  */
 sta_status sta_selftest_bounded_wait(uint64_t limit_ns, int32_t* dev_status, int32_t* waited_ok,
                                      sta_stream_t stream);
+
+/*
+ * Debug build (no counterpart on the pages; it stands in for a memory
+ * checker).  libsta_debug.so is this library compiled with STA_DEBUG=1 and
+ * exports the same calls.  Its kernels check every list entry, token index
+ * and TMEM column they touch; a failed check ORs STA_DEV_DEBUG into
+ * *dev_status and skips the access instead of trapping.  Results are those of
+ * the release build; the checks cost a few percent.
+ * sta_debug_build() returns 1 in libsta_debug.so and 0 in libsta.so.
+ */
+int sta_debug_build(void);
+
+/*
+ * Self-test of the debug build's index checks: one thread stores 1 into
+ * buf[index] through the checked path, where buf is a device int32 array of
+ * n elements (n >= 1).  An index outside [0, n) raises STA_DEV_DEBUG in
+ * *dev_status and stores nothing.  Only the debug build runs it: libsta.so
+ * has no checks and returns STA_ERR_UNSUPPORTED without launching anything.
+ * Errors: STA_ERR_ARG (null pointer, n < 1), STA_ERR_UNSUPPORTED, STA_ERR_CUDA.
+ */
+sta_status sta_selftest_index_check(int32_t* buf, int n, int index, int32_t* dev_status,
+                                    sta_stream_t stream);
 
 /* Library version (major*10000 + minor*100 + patch). */
 int sta_version(void);

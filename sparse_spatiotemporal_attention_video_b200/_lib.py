@@ -4,7 +4,11 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsta.so")
+# STA_LIB=debug selects libsta_debug.so, the build whose kernels check every
+# list entry, token index and TMEM column (build.py --debug)
+DEBUG_LIB_PATH = os.path.join(_HERE, "libsta_debug.so")
+LIB_PATH = DEBUG_LIB_PATH if os.environ.get("STA_LIB") == "debug" else os.path.join(
+    _HERE, "libsta.so")
 
 # sta_status
 STA_OK = 0
@@ -20,6 +24,7 @@ STA_DEV_CAPACITY = 0x2
 STA_DEV_EMPTY_ROW = 0x4
 STA_DEV_BAD_INDEX = 0x8
 STA_DEV_RANGE = 0x10
+STA_DEV_DEBUG = 0x20
 
 STA_BF16, STA_F32 = 0, 1
 (STA_SEL_RADIAL, STA_SEL_ENTROPY, STA_SEL_IBCS_SIP, STA_SEL_ROUTED, STA_SEL_TRA_TOKEN,
@@ -102,6 +107,9 @@ SIGNATURES = {
     "sta_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "sta_dev_status_string": (ctypes.c_char_p, [ctypes.c_int32]),
     "sta_version": (ctypes.c_int, []),
+    "sta_debug_build": (ctypes.c_int, []),
+    "sta_selftest_index_check": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_void_p, ctypes.c_void_p]),
     "sta_last_cuda_error": (ctypes.c_char_p, []),
     "sta_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint64, ctypes.c_void_p,
                                                  ctypes.c_void_p, ctypes.c_void_p]),
@@ -116,9 +124,10 @@ def load(path=LIB_PATH):
     if _lib is not None:
         return _lib
     if not os.path.exists(path):
+        flag = " --debug" if path == DEBUG_LIB_PATH else ""
         raise ImportError(
             f"{path} is missing: build it with "
-            "`python sparse_spatiotemporal_attention_video_b200/build.py` (nvcc, sm_100a)")
+            f"`python sparse_spatiotemporal_attention_video_b200/build.py{flag}` (nvcc, sm_100a)")
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():
         fn = getattr(lib, name)

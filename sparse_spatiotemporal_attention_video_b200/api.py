@@ -37,6 +37,19 @@ def sta_version():
     return _lib.load().sta_version()
 
 
+def sta_debug_build() -> bool:
+    """True when the loaded library is libsta_debug.so (STA_LIB=debug)."""
+    return bool(_lib.load().sta_debug_build())
+
+
+def sta_selftest_index_check(buf, n, index, dev_status, stream=None):
+    """Debug build: store 1 into buf[index] through the kernels' index check
+    (an index outside [0, n) raises STA_DEV_DEBUG and stores nothing)."""
+    lib = _lib.load()
+    check(lib.sta_selftest_index_check(_ptr(buf), int(n), int(index), _ptr(dev_status),
+                                       _stream(stream)), "sta_selftest_index_check")
+
+
 def sta_build_blocks_workspace(prob: Problem, sel: SelectorParams) -> int:
     return _lib.load().sta_build_blocks_workspace(ctypes.byref(prob), ctypes.byref(sel))
 

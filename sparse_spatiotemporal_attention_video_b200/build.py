@@ -1,10 +1,12 @@
 """Build libsta.so in-tree with nvcc for sm_100a.
 
-    python sparse_spatiotemporal_attention_video_b200/build.py [--verbose]
+    python sparse_spatiotemporal_attention_video_b200/build.py [--verbose] [--debug]
 
 Every .cu file under csrc/ is compiled to an object (in parallel), then
 linked into one shared library next to this file.  No torch types cross the
-library boundary, so no torch extension machinery is involved.
+library boundary, so no torch extension machinery is involved.  --debug
+builds libsta_debug.so instead: the same sources with STA_DEBUG=1, whose
+kernels check every list entry, token index and TMEM column they use.
 """
 import concurrent.futures
 import glob
@@ -17,6 +19,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libsta.so")
+OUT_DEBUG = os.path.join(PKG, "libsta_debug.so")
 BUILD = os.path.join(ROOT, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -31,8 +34,8 @@ def nvcc():
     raise RuntimeError("nvcc not found")
 
 
-def _compile(src, verbose, extra):
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+def _compile(src, verbose, extra, build_dir):
+    obj = os.path.join(build_dir, os.path.basename(src) + ".o")
     cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
         cmd += ["-Xptxas", "-v"]
@@ -42,23 +45,26 @@ def _compile(src, verbose, extra):
     return obj, r.stderr
 
 
-def build(verbose=False, extra=()):
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose=False, extra=(), debug=False):
+    build_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    out = OUT_DEBUG if debug else OUT
+    extra = list(extra) + (["-DSTA_DEBUG=1"] if debug else [])
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        results = list(ex.map(lambda s: _compile(s, verbose, list(extra)), srcs))
+        results = list(ex.map(lambda s: _compile(s, verbose, extra, build_dir), srcs))
     if verbose:
         for _, log in results:
             sys.stderr.write(log)
     objs = [o for o, _ in results]
-    tmp = OUT + ".tmp"
+    tmp = out + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, OUT)
-    return OUT
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(verbose="--verbose" in sys.argv))
+    print(build(verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

@@ -481,6 +481,7 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       tok = I.q_start + r;
     }
     bool active = tok >= 0;
+    if (active && !dcheck(tok < a.N, a.dev_status)) active = false;
     if (active && I.kind == kItemLocal && __ldg(a.routed_flag + tok)) active = false;
     const size_t orow = static_cast<size_t>(I.head) * a.N + (tok < 0 ? 0 : tok);
     if (I.ntiles == 0) {
@@ -518,6 +519,11 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       const uint32_t gg = g + t;
       const uint32_t sb = gg & 1;
       const uint32_t tS = tmem + lane_off + sb * 128;
+      if (!dcheck(tmem_in_range(tS + J * 64, tmem, 64) && tmem_in_range(tO, tmem, D),
+                  a.dev_status)) {
+        ok = false;
+        break;
+      }
       // Only the raw entries stay live across the tile; the per-slot masks
       // are derived from them on the (rare) masked path.
       HalfRaw<UNIT> raw = {};
@@ -718,6 +724,12 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         const float H = Z > 0.f ? logf(Z) - 0.6931471805599453f * (A / Z) : 0.f;
         a.entropy[orow] = H;
       }
+    }
+    if (!dcheck(tmem_in_range(tmem + lane_off + 256 + OB, tmem, OH) &&
+                    tmem_in_range(tmem + lane_off + 256 + D + OB, tmem, OH),
+                a.dev_status)) {
+      ok = false;
+      break;
     }
 #pragma unroll
     for (int ch = 0; ch < OH / 32; ++ch) {
@@ -962,7 +974,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool present = p_next;
             fetch(t + 1, e_next, p_next);
             // an out-of-range entry loads unit 0 (the softmax masks its slot)
-            const bool valid = present && e >= 0 && e < n_units;
+            const bool valid = present && e >= 0 && e < n_units &&
+                               dcheck(e * unit < a.N, a.dev_status);
             if (present && !valid && !is_v) raise_status(a.dev_status, STA_DEV_BAD_INDEX);
             u = valid ? e : 0;
           }
@@ -1064,6 +1077,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t sb = (g + t) & 1;
           const uint32_t tS = tmem + sb * 128;
+          // S buffer (128 columns) and O_1, the accumulator PV reaches last
+          if (!dcheck(tmem_in_range(tS, tmem, 128) && tmem_in_range(tmem + 256 + D, tmem, D),
+                      a.dev_status)) {
+            ok = false;
+            break;
+          }
           const uint32_t kbase = aK + st * L::TILE_BYTES;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {

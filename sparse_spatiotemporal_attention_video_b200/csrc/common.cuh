@@ -24,6 +24,32 @@ __device__ __forceinline__ void raise_status(int32_t* dev_status, int32_t bits) 
   if (dev_status) atomicOr(dev_status, bits);
 }
 
+// Index checks of the STA_DEBUG build (libsta_debug.so): dcheck(ok, st)
+// returns ok and, when ok is false, raises STA_DEV_DEBUG; the caller skips
+// the guarded access.  In the release build it is `true` and the condition
+// is compiled away.
+#ifndef STA_DEBUG
+#define STA_DEBUG 0
+#endif
+__device__ __forceinline__ bool dcheck(bool ok, int32_t* dev_status) {
+#if STA_DEBUG
+  if (!ok) raise_status(dev_status, STA_DEV_DEBUG);
+  return ok;
+#else
+  (void)ok;
+  (void)dev_status;
+  return true;
+#endif
+}
+// TMEM address (lane << 16 | column) of an access of `cols` columns by a
+// warp's 32 lanes inside the `alloc` columns allocated at `base`.
+__device__ __forceinline__ bool tmem_in_range(uint32_t addr, uint32_t base, uint32_t cols,
+                                              uint32_t alloc = 512) {
+  const uint32_t col = (addr & 0xffffu) - (base & 0xffffu);
+  const uint32_t lane = addr >> 16;
+  return col + cols <= alloc && lane + 32u <= 128u;
+}
+
 // Token layout of a sequence ("Token Radius Attention for Efficient Video
 // Generation", 2. Methodology, The TRA Pipeline, Efficient Execution: tokens
 // reordered tile by tile).  Within a frame, positions run over spatial tiles
@@ -189,6 +215,8 @@ cudaError_t launch_sip_sample(const float* p, int rows, int n_sub, int m, uint64
                               int32_t* required_cap, int32_t* dev_status, cudaStream_t s);
 
 // Self-test of the bounded wait (selftest.cu).
+cudaError_t launch_index_check_selftest(int32_t* buf, int n, int index, int32_t* dev_status,
+                                        cudaStream_t s);
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, int32_t* dev_status,
                                          int32_t* waited_ok, cudaStream_t s);
 

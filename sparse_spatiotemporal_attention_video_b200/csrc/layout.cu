@@ -46,7 +46,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_rows_kernel(
       const int kr = k + lane / vpr;  // this lane's row within the 32
       const int v = lane % vpr;
       const int t = __shfl_sync(0xffffffffu, tok, kr & 31);
-      if (kr < n) {
+      // (no status word here: a failed debug check only skips the row)
+      if (kr < n && dcheck(t >= 0 && t < rows, nullptr)) {
         const long long row = r0 + kr;
         const long long src = inverse ? row : t;
         const long long dst = inverse ? t : row;

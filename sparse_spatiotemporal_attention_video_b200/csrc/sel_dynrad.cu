@@ -191,7 +191,8 @@ __global__ void __launch_bounds__(kDynThreads) dynrad_lists_kernel(const DynArgs
     int pos = running;
     for (int w = 0; w < warp; ++w) pos += warp_tot[w];
     pos += __popc(bal & ((1u << lane) - 1u));
-    if (keep && pos < a.cap) out[pos] = cand[j];
+    if (keep && pos < a.cap && dcheck(cand[j] >= 0 && cand[j] < a.nb, a.dev_status))
+      out[pos] = cand[j];
     __syncthreads();
     if (threadIdx.x == 0)
       for (int w = 0; w < kDynThreads / 32; ++w) running += warp_tot[w];

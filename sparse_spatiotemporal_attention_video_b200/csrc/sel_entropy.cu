@@ -212,7 +212,7 @@ __global__ void __launch_bounds__(kRowWarps * 32) entropy_rows_kernel(const EntA
     }
     const unsigned bal = __ballot_sync(0xffffffffu, keep);
     const int pos = total + __popc(bal & ((1u << lane) - 1u));
-    if (keep && pos < a.cap) out[pos] = kb;
+    if (keep && pos < a.cap && dcheck(kb < nb, a.dev_status)) out[pos] = kb;
     total += __popc(bal);
   }
   if (lane == 0) {

@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kSipThreads, G <= 8 ? 4 : 1) sip_sample_kernel
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       if (bits & (1u << e)) {
-        if (pos < cap) {
+        if (pos < cap && dcheck(4 * (tid + k * kSipThreads) + e < n_sub, dev_status)) {
           out[pos] = 4 * (tid + k * kSipThreads) + e;
           if (lw) lw[pos] = -logf(pi_of(4 * k + e));
         }

@@ -196,6 +196,10 @@ __global__ void __launch_bounds__(kImpTcThreads, 1)
         }
         tc_fence_after();
         const uint32_t tAcc = tmem + acc * kImpTile;
+        if (!dcheck(tmem_in_range(tAcc, tmem, kImpTile, 2 * kImpTile), a.dev_status)) {
+          ok = false;
+          break;
+        }
         const uint32_t bH = bBase + st * 2 * kImpTileBytes, bL = bH + kImpTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -245,6 +249,10 @@ __global__ void __launch_bounds__(kImpTcThreads, 1)
       {
         uint32_t v0[32], v1[32];
         const uint32_t ta = tmem + lane_off + acc * kImpTile + J * 64;
+        if (!dcheck(tmem_in_range(ta, tmem, 64, 2 * kImpTile), a.dev_status)) {
+          ok = false;
+          break;
+        }
         tmem_ld32(ta, v0);
         tmem_ld32(ta + 32, v1);
         tmem_wait_ld();

@@ -86,7 +86,8 @@ __global__ void __launch_bounds__(kThreads) radial_lists_kernel(
     int before = running;
     for (int w = 0; w < warp; ++w) before += warp_counts[w];
     const int pos = before + __popc(ballot & ((1u << lane) - 1u));
-    if (keep && pos < cap) idx[static_cast<size_t>(qb) * cap + pos] = kb;
+    if (keep && pos < cap && dcheck(kb < nb && qb < nb, dev_status))
+      idx[static_cast<size_t>(qb) * cap + pos] = kb;
     __syncthreads();
     if (threadIdx.x == 0) {
       int tot = 0;

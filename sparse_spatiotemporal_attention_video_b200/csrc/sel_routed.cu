@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(256) routed_local_lists_kernel(
     }
     const unsigned bal = __ballot_sync(0xffffffffu, keep);
     const int pos = total + __popc(bal & ((1u << lane) - 1u));
-    if (keep && pos < cap) out[pos] = u;
+    if (keep && pos < cap && dcheck(u * U < N, dev_status)) out[pos] = u;
     total += __popc(bal);
   }
   if (lane == 0) {

@@ -99,6 +99,11 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
     const int t = q0 + r;  // sequence position
     int f, h, w, run;
     layout_coords(a.L, t, f, h, w, run);
+    if (!dcheck(f < a.F && h < a.H && w < a.W, a.dev_status)) {
+      qr0[r] = 0.f;  // the query is dropped (it reaches no key)
+      qf[r] = qh[r] = qw[r] = 0;
+      continue;
+    }
     qf[r] = f;
     qh[r] = h;
     qw[r] = w;
@@ -221,7 +226,7 @@ __global__ void __launch_bounds__(kTraThreads) tra_token_lists_kernel(const TraA
     int pos = before + inc - cntw;
     for (uint32_t b = bits; b; b &= b - 1u) {
       const int kb = c0 + threadIdx.x * 32 + (__ffs(b) - 1);
-      if (pos < a.cap) out[pos] = kb;
+      if (pos < a.cap && dcheck(kb < a.nb, a.dev_status)) out[pos] = kb;
       ++pos;
     }
     __syncthreads();

@@ -9,6 +9,8 @@
 
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 using namespace sta;
@@ -19,6 +21,16 @@ constexpr int kVersion = 200;  // 0.2.0 (selector parameters gained the token la
 
 // Last CUDA error a call of this thread ran into (sta_last_cuda_error).
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+// An NVTX range named after the entry point, around each call that enqueues
+// selector or attention work (recorded by profilers that trace NVTX, e.g.
+// `ncu --nvtx --nvtx-include "sta_sparse_attn_fwd/"`; a no-op otherwise).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 bool failed(cudaError_t e) {
   if (e == cudaSuccess) return false;
@@ -227,6 +239,19 @@ extern "C" {
 
 int sta_version(void) { return kVersion; }
 
+int sta_debug_build(void) { return STA_DEBUG ? 1 : 0; }
+
+sta_status sta_selftest_index_check(int32_t* buf, int n, int index, int32_t* dev_status,
+                                    sta_stream_t stream) {
+  if (!buf || !dev_status || n < 1) return STA_ERR_ARG;
+  // without the checks an out-of-range index would be stored as given
+  if (!STA_DEBUG) return STA_ERR_UNSUPPORTED;
+  if (failed(launch_index_check_selftest(buf, n, index, dev_status,
+                                         reinterpret_cast<cudaStream_t>(stream))))
+    return STA_ERR_CUDA;
+  return STA_OK;
+}
+
 sta_status sta_selftest_bounded_wait(uint64_t limit_ns, int32_t* dev_status, int32_t* waited_ok,
                                      sta_stream_t stream) {
   if (!dev_status || !waited_ok) return STA_ERR_ARG;
@@ -255,6 +280,7 @@ const char* sta_status_string(sta_status s) {
 
 const char* sta_dev_status_string(int32_t bits) {
   if (bits == 0) return "ok";
+  if (bits & STA_DEV_DEBUG) return "debug build: an index check failed (access skipped)";
   if (bits & STA_DEV_TIMEOUT) return "timeout: a bounded wait ran out";
   if (bits & STA_DEV_BAD_INDEX) return "list entry out of range (skipped)";
   if (bits & STA_DEV_RANGE) return "importance operand beyond the fp16 range";
@@ -289,6 +315,7 @@ size_t sta_build_blocks_workspace(const sta_problem* prob, const sta_selector_pa
 sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* sel,
                             const void* q, const void* k, sta_block_lists* out, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  NvtxRange nvtx_range("sta_build_blocks");
   sta_status st = check_problem(prob);
   if (st != STA_OK) return st;
   if (!sel || !out || !out->idx || !out->cnt || out->cap < 1) return STA_ERR_ARG;
@@ -505,6 +532,7 @@ sta_status sta_sparse_attn_fwd(const sta_problem* prob, const sta_attn_params* p
                                const void* q, const void* k, const void* v,
                                const sta_block_lists* lists, void* o, void* workspace,
                                size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  NvtxRange nvtx_range("sta_sparse_attn_fwd");
   sta_status st = check_sparse_args(prob, prm, q, k, v, lists, o);
   if (st != STA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -592,6 +620,7 @@ sta_status dense_attn(const sta_problem* prob, const void* q, const void* k, con
 sta_status sta_dense_attn_fwd(const sta_problem* prob, const void* q, const void* k,
                               const void* v, float scale, void* o, void* workspace,
                               size_t workspace_bytes, int32_t* dev_status, sta_stream_t stream) {
+  NvtxRange nvtx_range("sta_dense_attn_fwd");
   return dense_attn(prob, q, k, v, scale, o, nullptr, workspace, workspace_bytes, dev_status,
                     stream);
 }
@@ -600,6 +629,7 @@ sta_status sta_dense_attn_entropy_fwd(const sta_problem* prob, const void* q, co
                                       const void* v, float scale, void* o, float* entropy,
                                       void* workspace, size_t workspace_bytes,
                                       int32_t* dev_status, sta_stream_t stream) {
+  NvtxRange nvtx_range("sta_dense_attn_entropy_fwd");
   if (!entropy) return STA_ERR_ARG;
   return dense_attn(prob, q, k, v, scale, o, entropy, workspace, workspace_bytes, dev_status,
                     stream);
@@ -607,6 +637,7 @@ sta_status sta_dense_attn_entropy_fwd(const sta_problem* prob, const void* q, co
 
 sta_status sta_permute_tokens(const sta_problem* prob, int tile_h, int tile_w, int inverse,
                               const void* in, void* out, sta_stream_t stream) {
+  NvtxRange nvtx_range("sta_permute_tokens");
   sta_status st = check_problem(prob);
   if (st != STA_OK) return st;
   if (!in || !out || tile_h < 1 || tile_w < 1 || tile_h > prob->H || tile_w > prob->W)
