@@ -7,7 +7,7 @@
 // with s_ik = scale * q_i.k_k; keys outside the listed units never enter the
 // softmax; w_k = 1/pi of the key's sampled unit (stored as -ln pi) or 1.
 //
-// How (one persistent CTA per SM, 10 warps):
+// How (one persistent CTA per SM, 12 warps):
 //   warp 0      producer: TMA loads of the 128-row Q tile and, per 128-key
 //               tile, of the listed key/value units (kv_unit rows each,
 //               128-byte swizzle) into a K ring and a V ring; gathered query
@@ -17,12 +17,17 @@
 //               out [8-row group][half][8 rows][128 B]: a 128-key tile then
 //               takes 8 copies per operand instead of 16 of 2 KB, which the
 //               copy engine serves too slowly to keep the tensor core busy.
-//   warp 1      MMA issuer (one thread): S = Q K^T of tile t into TMEM S
+//   warp 1      QK issuer (one thread): S = Q K^T of tile t into TMEM S
 //               buffer t%2 (tcgen05.mma, M=128 N=128 K=16 steps, both
-//               operands K-major in shared memory), then O_0 += P[:, 0:64]
-//               V[0:64] and O_1 += P[:, 64:128] V[64:128] with P read from
-//               TMEM (bf16, aliased onto the S buffer) and V MN-major in
-//               shared memory.  QK of tile t+1 is issued before PV of tile t.
+//               operands K-major in shared memory), once the PV of tile t-2
+//               (which reads P from that buffer) has completed.
+//   warp 11     PV issuer (one thread): O_0 += P[:, 0:64] V[0:64] and
+//               O_1 += P[:, 64:128] V[64:128] with P read from TMEM (bf16,
+//               aliased onto the S buffer) and V MN-major in shared memory.
+//               The two issuers feed one tensor pipe: while one waits on a
+//               barrier or commits, the other's products keep it busy (one
+//               thread issuing both streams left the pipe idle for about
+//               800 cycles per tile).
 //               TMEM: S_0 | S_1 | O_0 | O_1 (512 columns).
 //   warps 2-9   softmax, two groups of 4 warps.  Group J owns keys
 //               [64J, 64J+64) of every tile and the accumulator O_J: thread r
@@ -56,10 +61,11 @@
 namespace sta {
 namespace {
 
-// Warp 0 Q/K producer, warp 1 MMA issuer, warps 2-9 two softmax groups,
-// warp 10 V producer.
+// Warp 0 Q/K producer, warp 1 QK issuer, warps 2-9 two softmax groups,
+// warp 10 V producer, warp 11 PV issuer.
 constexpr int kWarpV = 10;
-constexpr int kThreads = 352;
+constexpr int kWarpPV = 11;
+constexpr int kThreads = 384;
 constexpr int kHalfBytes = 128 * 128;  // 128 rows x 128 bytes: one 64-column half of a tile
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -847,7 +853,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(o_done + i, 1);
     }
     mbar_init(o_free, 8);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);  // one commit from each issuer
     for (int i = 0; i < 4; ++i) mbar_init(lbar + i, 2);
     *abort = 0;
     fence_barrier_init();
@@ -1007,56 +1013,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(ring_full + (i % RS), (i / RS) & 1, no_abort, limit);
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+    // ----------------------------------------------------------- QK issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-      uint32_t kt = 0, vt = 0, qn = 0, g = 0;
+      const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+      uint32_t kt = 0, qn = 0, g = 0;
       bool ok = true;
-      // first: the next PV starts the accumulators O_0 / O_1 of this item.
-      // O_0/O_1 stay in use until both softmax groups have finished the
-      // item's epilogue (o_free, one phase per item): nfree counts the
-      // phases seen.  The first PV of item qn waits for epilogues 0..qn-1.
-      bool first = true;
-      uint32_t nfree = 0;
-      auto ensure_free = [&](uint32_t k) -> bool {
-        while (nfree < k) {
-          if (!mbar_wait(o_free, nfree & 1, abort, limit)) return false;
-          ++nfree;
-        }
-        return true;
-      };
-      // K/V tiles of the current item are in the interleaved layout: 8-row
-      // groups 2048 bytes apart, halves 1024 apart (else 1024 and 16384)
-      bool il = false;
-      auto issue_pv = [&](uint32_t gg) -> bool {
-        const uint32_t sb = gg & 1;
-        if (!mbar_wait(p_full + sb, (gg >> 1) & 1, abort, limit)) return false;
-        if (first && !ensure_free(qn)) return false;
-        tc_fence_after();
-        const int st = vt % VS;
-        if (!mbar_wait(v_full + st, (vt / VS) & 1, abort, limit)) return false;
-        tc_fence_after();
-        const uint32_t tS = tmem + sb * 128;
-        const uint32_t vbase = aV + st * L::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < kTileK / 16; ++kk) {
-          // V is MN-major: LBO steps between the two 64-column halves, SBO
-          // between the two 8-key groups of the 16-key step
-          const uint64_t bdesc = il ? smem_desc_sw128(vbase + kk * 4096, 1024, 2048)
-                                    : smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024);
-          // keys 0..63 (softmax group 0): P in columns 0..31, into O_0;
-          // keys 64..127 (group 1): P in columns 64..95, into O_1
-          const uint32_t pa = tS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
-          const uint32_t tO = tmem + 256 + (kk < 4 ? 0 : D);
-          mma_bf16_ts(tO, pa, bdesc, IDESC_PV, (first && (kk & 3) == 0) ? 0u : 1u);
-        }
-        first = false;
-        ++vt;
-        mma_commit(o_done + sb);
-        return true;
-      };
       for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
         if (*abort) break;
         const Item I = decode_item(a, it);
@@ -1065,21 +1027,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        tc_fence_after();
-        first = true;
-        il = kInterleaved && (I.kind == kItemList || I.kind == kItemLocal);
+        // K tiles of the current item are in the interleaved layout: 8-row
+        // groups 2048 bytes apart, halves 1024 apart (else 1024 and 16384)
+        const bool il = kInterleaved && (I.kind == kItemList || I.kind == kItemLocal);
         for (int t = 0; t < I.ntiles; ++t) {
+          const uint32_t gg = g + t;
+          const uint32_t sb = gg & 1;
           const int st = kt % KS;
           if (!mbar_wait(k_full + st, (kt / KS) & 1, abort, limit)) {
             ok = false;
             break;
           }
+          // S buffer sb holds P of tile gg - 2 until the PV that reads it
+          // has completed (the PV issuer commits o_done[sb] after it; that
+          // PV cannot complete twice before this QK, which its successor
+          // needs, is issued)
+          if (gg >= 2 && !mbar_wait(o_done + sb, ((gg - 2) >> 1) & 1, abort, limit)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          const uint32_t sb = (g + t) & 1;
           const uint32_t tS = tmem + sb * 128;
-          // S buffer (128 columns) and O_1, the accumulator PV reaches last
-          if (!dcheck(tmem_in_range(tS, tmem, 128) && tmem_in_range(tmem + 256 + D, tmem, D),
-                      a.dev_status)) {
+          if (!dcheck(tmem_in_range(tS, tmem, 128), a.dev_status)) {
             ok = false;
             break;
           }
@@ -1096,21 +1065,82 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++kt;
           mma_commit(s_full + sb);
           if (t == I.ntiles - 1) mma_commit(q_empty);
-          if (t > 0 && !issue_pv(g + t - 1)) {
-            ok = false;
-            break;
-          }
         }
         if (!ok) break;
-        if (!issue_pv(g + I.ntiles - 1)) {
-          ok = false;
-          break;
-        }
         ++qn;
         g += I.ntiles;
       }
       if (!ok) fail(abort, a.dev_status);
-      // all issued MMAs complete before TMEM is released
+      // all issued MMAs (of both issuers) complete before TMEM is released
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0, no_abort, limit);
+    }
+    __syncwarp();
+  } else if (warp == kWarpPV) {
+    // ----------------------------------------------------------- PV issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t aV = smem_u32(sV);
+      uint32_t vt = 0, qn = 0, g = 0;
+      bool ok = true;
+      // O_0/O_1 stay in use until both softmax groups have finished the
+      // item's epilogue (o_free, one phase per item): nfree counts the
+      // phases seen.  The first PV of item qn waits for epilogues 0..qn-1.
+      uint32_t nfree = 0;
+      auto ensure_free = [&](uint32_t k) -> bool {
+        while (nfree < k) {
+          if (!mbar_wait(o_free, nfree & 1, abort, limit)) return false;
+          ++nfree;
+        }
+        return true;
+      };
+      for (int it = blockIdx.x; it < a.n_items && ok; it += gridDim.x) {
+        if (*abort) break;
+        const Item I = decode_item(a, it);
+        if (I.ntiles == 0) continue;
+        // V tiles in the interleaved layout as the K tiles above
+        const bool il = kInterleaved && (I.kind == kItemList || I.kind == kItemLocal);
+        for (int t = 0; t < I.ntiles; ++t) {
+          const uint32_t gg = g + t;
+          const uint32_t sb = gg & 1;
+          if (!mbar_wait(p_full + sb, (gg >> 1) & 1, abort, limit) ||
+              (t == 0 && !ensure_free(qn))) {
+            ok = false;
+            break;
+          }
+          const int st = vt % VS;
+          if (!mbar_wait(v_full + st, (vt / VS) & 1, abort, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t tS = tmem + sb * 128;
+          // O_1, the accumulator PV reaches last
+          if (!dcheck(tmem_in_range(tmem + 256 + D, tmem, D), a.dev_status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t vbase = aV + st * L::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kTileK / 16; ++kk) {
+            // V is MN-major: LBO steps between the two 64-column halves, SBO
+            // between the two 8-key groups of the 16-key step
+            const uint64_t bdesc = il ? smem_desc_sw128(vbase + kk * 4096, 1024, 2048)
+                                      : smem_desc_sw128(vbase + kk * 2048, kHalfBytes, 1024);
+            // keys 0..63 (softmax group 0): P in columns 0..31, into O_0;
+            // keys 64..127 (group 1): P in columns 64..95, into O_1
+            const uint32_t pa = tS + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+            const uint32_t tO = tmem + 256 + (kk < 4 ? 0 : D);
+            mma_bf16_ts(tO, pa, bdesc, IDESC_PV, (t == 0 && (kk & 3) == 0) ? 0u : 1u);
+          }
+          ++vt;
+          mma_commit(o_done + sb);
+        }
+        if (!ok) break;
+        ++qn;
+        g += I.ntiles;
+      }
+      if (!ok) fail(abort, a.dev_status);
       mma_commit(mma_done);
       mbar_wait(mma_done, 0, no_abort, limit);
     }
