@@ -34,7 +34,7 @@
 //               of the group holds query row r (TMEM lane r), reads its 64
 //               logits, masks partial units / the local window, adds
 //               log-weights, keeps its own running max m_J and sum l_J in
-//               registers (max updates that move by <= 8 in log2 units are
+//               registers (max updates that move by <= 16 in log2 units are
 //               deferred, so O_J is rescaled only on large jumps) and writes
 //               P as bf16 into TMEM.  The two groups never wait on each other
 //               inside an item: each is an independent online softmax over its
@@ -71,9 +71,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // Tuning constants (compile-time).
 // Deferred rescale: the running row maximum moves (and O is rescaled) only
-// when a tile's maximum exceeds it by more than this many log2 units.
+// when a tile's maximum exceeds it by more than this many log2 units.  P
+// then stays below 2^16 (bf16 and the fp32 sums have the range to spare);
+// 16 measured 2% faster than 8 on every workload (fewer waits for the
+// previous tile's PV before a rescale).
 #ifndef STA_RESCALE_THRESHOLD
-#define STA_RESCALE_THRESHOLD 8.0f
+#define STA_RESCALE_THRESHOLD 16.0f
 #endif
 constexpr float kRescaleThreshold = STA_RESCALE_THRESHOLD;
 // Speculative row maximum (see softmax_role); 0 finds each tile's maximum
@@ -277,13 +280,52 @@ __device__ __forceinline__ void half_info_from_raw(const AttnArgs& a, const Item
   }
 }
 
+// The local window of one query row ("Where Compute Matters: Heterogeneous
+// Attention for Efficient Video Diffusion", Abstract: easy tokens attend to a
+// spatiotemporal neighbourhood): key (f, h, w) is inside iff |f - fq| <=
+// win_f, -win_h <= h - hq < win_h and -win_w <= w - wq < win_w, with
+// (fq, hq, wq) the query's grid position.
+struct WinGeom {
+  int fq, hq, wq;
+};
+
+// Bit c (c < n <= 64) set iff the key c places after grid position (f, h,
+// w) in raster order lies in the window.  The keys are walked as runs
+// within one grid row, one column interval per run: a run ends at the row's
+// end, so a slot of n <= W keys is one or two runs.
+__device__ __forceinline__ uint64_t window_bits(int f, int h, int w, int n, const AttnArgs& a,
+                                                const WinGeom& g) {
+  uint64_t bits = 0;
+  for (int c0 = 0; c0 < n;) {
+    const int run = min(a.W - w, n - c0);
+    const int df = f - g.fq, dh = h - g.hq;
+    if (df <= a.win_f && df >= -a.win_f && dh >= -a.win_h && dh < a.win_h) {
+      // run columns [lo, hi): keys w + lo .. w + hi - 1 of this row
+      const int lo = max(g.wq - a.win_w - w, 0);
+      const int hi = min(g.wq + a.win_w - w, run);
+      if (hi > lo) {
+        const int len = hi - lo;
+        const uint64_t ones = len >= 64 ? ~0ull : ((1ull << len) - 1ull);
+        bits |= ones << (c0 + lo);
+      }
+    }
+    c0 += run;
+    w = 0;
+    if (++h == a.H) {
+      h = 0;
+      ++f;
+    }
+  }
+  return bits;
+}
+
 // Masks (partial units, key tokens past N) and the local window on one
 // group's 64 logit columns.  Log-weights are not added here: they are
 // constant per slot, so the caller folds them into the per-slot maxima and
 // into the exponent's offset.
 template <int UNIT>
 __device__ __forceinline__ void mask_half(float (&x)[64], const HalfInfo<UNIT>& hi, bool window,
-                                          const AttnArgs& a, int fq, int hq, int wq) {
+                                          const uint64_t* wbits) {
   constexpr int W = HalfInfo<UNIT>::W;
   if (!hi.full) {
 #pragma unroll
@@ -291,42 +333,14 @@ __device__ __forceinline__ void mask_half(float (&x)[64], const HalfInfo<UNIT>& 
       if ((c % W) >= hi.lim[c / W]) x[c] = -INFINITY;
   }
   if (window) {
-    // Per slot: when the slot's W keys lie in one grid row (same f and h),
-    // the window is one column interval [lo, hi) of the slot; otherwise the
-    // key coordinates are walked column by column.
-    const int S = a.H * a.W;
+    // Per slot: the bit set of the columns whose keys lie in the query's
+    // window (window_bits, formed by the caller), applied column by column.
 #pragma unroll
     for (int sl = 0; sl < HalfInfo<UNIT>::SLOTS; ++sl) {
-      const int t0 = hi.tok0[sl];
-      int f = t0 / S;
-      const int rem = t0 - f * S;
-      int h = rem / a.W;
-      int w = rem - h * a.W;
-      if (w + W <= a.W) {
-        const int df = f - fq, dh = h - hq;
-        const bool row_in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
-                            (dh < a.win_h);
-        const int lo = row_in ? wq - a.win_w - w : W;
-        const int hi_c = row_in ? wq + a.win_w - w : 0;
+      const uint64_t bits = wbits[sl];
 #pragma unroll
-        for (int c = 0; c < W; ++c)
-          if (c < lo || c >= hi_c) x[sl * W + c] = -INFINITY;
-      } else {
-#pragma unroll
-        for (int c = 0; c < W; ++c) {
-          const int df = f - fq, dh = h - hq, dw = w - wq;
-          const bool in = (df <= a.win_f) && (df >= -a.win_f) && (dh >= -a.win_h) &&
-                          (dh < a.win_h) && (dw >= -a.win_w) && (dw < a.win_w);
-          if (!in) x[sl * W + c] = -INFINITY;
-          if (++w == a.W) {
-            w = 0;
-            if (++h == a.H) {
-              h = 0;
-              ++f;
-            }
-          }
-        }
-      }
+      for (int c = 0; c < W; ++c)
+        if (!((bits >> c) & 1ull)) x[sl * W + c] = -INFINITY;
     }
   }
 }
@@ -450,7 +464,7 @@ __device__ __forceinline__ void load_cols64(uint32_t taddr, float (&x)[64]) {
 // Softmax warpgroup J (4 warps): keys [64J, 64J+64) of every tile, query
 // row r = 32*quadrant + lane per thread, accumulator O_J (see the file
 // comment).
-template <int D, int UNIT, bool ENT>
+template <int D, int UNIT, bool ENT, bool WIN>
 __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxShared& sh,
                                              uint32_t tmem, int warp, int lane, int J) {
   constexpr int OH = D / 2;     // output columns per group
@@ -504,14 +518,15 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
       }
       continue;
     }
-    int fq = 0, hq = 0, wq = 0;
-    const bool window = (I.kind == kItemLocal);
+    // the local-window code exists only in the routed kernels (WIN)
+    const bool window = WIN && (I.kind == kItemLocal);
+    WinGeom wg{0, 0, 0};
     if (window && tok >= 0) {
       const int S = a.H * a.W;
-      fq = tok / S;
-      const int rem = tok - fq * S;
-      hq = rem / a.W;
-      wq = rem - hq * a.W;
+      wg.fq = tok / S;
+      const int rem = tok - wg.fq * S;
+      wg.hq = rem / a.W;
+      wg.wq = rem - wg.hq * a.W;
     }
     const bool dense_like = (I.kind == kItemDense || I.kind == kItemGatherDense);
     const bool weighted = !dense_like && a.logw != nullptr;
@@ -545,6 +560,32 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         load_half_raw<UNIT>(a, I, t + 1, J, raw_next);  // next tile's entries
       }
       const bool simple = full && !weighted && !window;  // no mask, no weight
+      constexpr int SW = HalfInfo<UNIT>::W, NS = HalfInfo<UNIT>::SLOTS;
+      // Local items: this row's window columns of each slot.  The grid
+      // position of slot q's first key is the same for every row: lane q
+      // forms it (one division sequence for all slots) and the warp reads
+      // it by shuffle; each row then walks the slot's row runs.
+      uint64_t wbits[NS];
+      if (window) {
+        int t0_mine = 0;
+#pragma unroll
+        for (int q = 0; q < NS; ++q) {
+          const int col = J * 64 + q * SW;
+          const int u = static_cast<unsigned>(raw.u[q]) < static_cast<unsigned>(n_units)
+                            ? raw.u[q] : 0;
+          if (lane == q) t0_mine = u * UNIT + (col - (col / UNIT) * UNIT);
+        }
+        const int S = a.H * a.W;
+        const int f_m = t0_mine / S;
+        const int rem = t0_mine - f_m * S;
+        const int h_m = rem / a.W;
+        const int w_m = rem - h_m * a.W;
+#pragma unroll
+        for (int q = 0; q < NS; ++q)
+          wbits[q] = window_bits(__shfl_sync(0xffffffffu, f_m, q),
+                                 __shfl_sync(0xffffffffu, h_m, q),
+                                 __shfl_sync(0xffffffffu, w_m, q), SW, a, wg);
+      }
       if (!__all_sync(0xffffffffu,
                       mbar_wait(sh.s_full + sb, (gg >> 1) & 1, abort, limit))) {
         ok = false;
@@ -557,16 +598,15 @@ __device__ __forceinline__ void softmax_role(const AttnArgs& a, const SoftmaxSha
         if (dense_like) {
           HalfInfo<kTileK> td;
           load_half_info<kTileK>(a, I, t, J, inv_scale, td);  // geometry only, no loads
-          mask_half<kTileK>(x, td, false, a, 0, 0, 0);
+          mask_half<kTileK>(x, td, false, nullptr);
         } else {
           HalfInfo<UNIT> ti;
           half_info_from_raw<UNIT>(a, I, J, inv_scale, raw, ti);
-          mask_half<UNIT>(x, ti, window, a, fq, hq, wq);
+          mask_half<UNIT>(x, ti, window, wbits);
         }
       }
       // per-slot log-weights (raw logit units), 0 without weights (a masked
       // slot's value does not matter: its logits are -inf)
-      constexpr int SW = HalfInfo<UNIT>::W, NS = HalfInfo<UNIT>::SLOTS;
       float bias[NS];
 #pragma unroll
       for (int q = 0; q < NS; ++q)
@@ -798,7 +838,7 @@ __device__ __forceinline__ void load_unit_il(uint8_t* tile, const CUtensorMap* m
   }
 }
 
-template <int D, int KS, int VS, int UNIT, bool ENT>
+template <int D, int KS, int VS, int UNIT, bool ENT, bool WIN>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k_u,
@@ -1149,7 +1189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------- softmax
     SoftmaxShared sh{s_full, p_full, o_done, o_free, lbar, abort};
     // one copy of the softmax code serves both groups (J is a runtime value)
-    softmax_role<D, UNIT, ENT>(a, sh, tmem, warp, lane, warp < 6 ? 0 : 1);
+    softmax_role<D, UNIT, ENT, WIN>(a, sh, tmem, warp, lane, warp < 6 ? 0 : 1);
   }
 
   tc_fence_before();
@@ -1167,14 +1207,14 @@ __global__ void f32_to_bf16_kernel(const float4* __restrict__ src, uint2* __rest
   }
 }
 
-template <int D, int KS, int VS, int UNIT, bool ENT = false>
+template <int D, int KS, int VS, int UNIT, bool ENT = false, bool WIN = false>
 cudaError_t launch_t(const AttnArgs& a, const CUtensorMap& tq, const CUtensorMap& tku,
                      const CUtensorMap& tvu, const CUtensorMap& tkf, const CUtensorMap& tvf,
                      const CUtensorMap& tki, const CUtensorMap& tvi, int num_sms,
                      cudaStream_t stream) {
   using L = Layout<D, KS, VS>;
-  auto kern = attn_fwd_kernel<D, KS, VS, UNIT, ENT>;
-  cudaError_t e = set_dyn_smem<attn_fwd_kernel<D, KS, VS, UNIT, ENT>>(L::ALLOC);
+  auto kern = attn_fwd_kernel<D, KS, VS, UNIT, ENT, WIN>;
+  cudaError_t e = set_dyn_smem<attn_fwd_kernel<D, KS, VS, UNIT, ENT, WIN>>(L::ALLOC);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
   if (grid <= 0) return cudaSuccess;
@@ -1200,10 +1240,15 @@ cudaError_t launch_attention(int d, const AttnArgs& a, const CUtensorMap& tq,
                                                                tvi, num_sms, stream);
     return cudaErrorInvalidValue;
   }
-#define STA_ATTN_CASE(DD, UU)                                                              \
-  if (d == DD && a.unit == UU)                                                             \
-    return launch_t<DD, STA_KSTAGES, STA_VSTAGES, UU>(a, tq, tku, tvu, tkf, tvf, tki, tvi, \
-                                                      num_sms, stream);
+  // routed lists (local windows) run their own instantiation, so that the
+  // window code costs the other kernels nothing
+  const bool routed = (a.mode == kModeRouted);
+#define STA_ATTN_CASE(DD, UU)                                                                \
+  if (d == DD && a.unit == UU)                                                               \
+    return routed ? launch_t<DD, STA_KSTAGES, STA_VSTAGES, UU, false, true>(                 \
+                        a, tq, tku, tvu, tkf, tvf, tki, tvi, num_sms, stream)                \
+                  : launch_t<DD, STA_KSTAGES, STA_VSTAGES, UU, false, false>(                \
+                        a, tq, tku, tvu, tkf, tvf, tki, tvi, num_sms, stream);
   STA_ATTN_CASE(128, 128)
   STA_ATTN_CASE(128, 64)
   STA_ATTN_CASE(128, 32)
