@@ -384,7 +384,7 @@ def config_of(w):
 
 
 # ------------------------------------------------------------------- GPU arm
-SELECTOR_LAUNCHES = {"radial": 1, "entropy": 3, "routed": 2, "ibcs_sip": 6, "tra_token": 1,
+SELECTOR_LAUNCHES = {"radial": 1, "entropy": 3, "routed": 2, "ibcs_sip": 4, "tra_token": 1,
                      "dynrad": 3}
 
 

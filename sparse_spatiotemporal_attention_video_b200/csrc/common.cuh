@@ -161,9 +161,13 @@ cudaError_t set_dyn_smem(int bytes) {
 }
 
 // Block means (sel_pool.cu): out_i[h][b][d] = mean of the rows of block b of
-// x_i (fp32); x1/out1 may be null.
+// x_i (fp32); x1/out1 may be null.  The _f16x2 form writes each mean as the
+// fp16 pair hi = fp16(m), lo = fp16(m - hi) instead (STA_DEV_RANGE beyond
+// the fp16 range).
 cudaError_t launch_block_means(const __nv_bfloat16* x0, const __nv_bfloat16* x1, float* out0,
                                float* out1, int heads, int N, int d, int U, cudaStream_t s);
+cudaError_t launch_block_means_f16x2(const __nv_bfloat16* x, __half* hi, __half* lo, int heads,
+                                     int N, int d, int U, int32_t* dev_status, cudaStream_t s);
 
 // Entropy-radius selector (sel_entropy.cu).
 int entropy_max_blocks(int d);
@@ -201,10 +205,9 @@ cudaError_t launch_routed_local_lists(int F, int H, int W, int B, int U, int win
 // Clustering importance + inclusion-probability sampling (sel_ibcs.cu,
 // sel_importance.cu).
 int ibcs_max_subblocks();
-cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
-                          int d, int B, int km_k, int iters, cudaStream_t s);
-cudaError_t launch_split_f16(const float* x, __half* hi, __half* lo, size_t n,
-                             int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_kmeans(const __nv_bfloat16* q, __half* cent_hi, __half* cent_lo, float* wts,
+                          int heads, int N, int d, int B, int km_k, int iters,
+                          int32_t* dev_status, cudaStream_t s);
 cudaError_t launch_importance_tc(const float* wts, float* p, int heads, int n_rows, int nqb,
                                  int km, int n_sub, int N, int U, float scale,
                                  const CUtensorMap& ch,

@@ -9,6 +9,7 @@
 // count (the last block of a head may be partial).
 #pragma once
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace sta {
@@ -36,12 +37,17 @@ __device__ __forceinline__ void pool_add_bf16x8(float (&acc)[8], const uint4 v) 
 }
 
 // Means of blocks first_unit .. first_unit + UPC - 1 (unit = head * nb + b)
-// of x [heads][N][D] into out [heads][nb][D].  part: 256 x 9 floats of shared
-// memory; the caller synchronises the CTA before reusing it.
+// of x [heads][N][D] into out [heads][nb][D] (fp32), or, when out is null,
+// as the fp16 pair hi = fp16(mean), lo = fp16(mean - hi) into hi/lo (the
+// tensor-core operands of the importance scores; a mean beyond the fp16
+// range sets *range_bad).  part: 256 x 9 floats of shared memory; the caller
+// synchronises the CTA before reusing it.
 template <int D, int U>
 __device__ __forceinline__ void pool_pass(const __nv_bfloat16* __restrict__ x,
                                           float* __restrict__ out, int heads, int N,
-                                          long long first_unit, float (*part)[9]) {
+                                          long long first_unit, float (*part)[9],
+                                          __half* hi = nullptr, __half* lo = nullptr,
+                                          bool* range_bad = nullptr) {
   using S = PoolShape<D, U>;
   const int nb = (N + U - 1) / U;
   const int tid = threadIdx.x;
@@ -83,9 +89,28 @@ __device__ __forceinline__ void pool_pass(const __nv_bfloat16* __restrict__ x,
       for (int i = 0; i < 8; ++i) s[i] += part[t][i];
     }
     const float inv = 1.0f / static_cast<float>(n);
-    float4* o = reinterpret_cast<float4*>(out + static_cast<size_t>(unit) * D + cg * 8);
-    o[0] = make_float4(s[0] * inv, s[1] * inv, s[2] * inv, s[3] * inv);
-    o[1] = make_float4(s[4] * inv, s[5] * inv, s[6] * inv, s[7] * inv);
+    if (out) {
+      float4* o = reinterpret_cast<float4*>(out + static_cast<size_t>(unit) * D + cg * 8);
+      o[0] = make_float4(s[0] * inv, s[1] * inv, s[2] * inv, s[3] * inv);
+      o[1] = make_float4(s[4] * inv, s[5] * inv, s[6] * inv, s[7] * inv);
+    } else {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float v0 = s[2 * i] * inv, v1 = s[2 * i + 1] * inv;
+        const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
+        const __half l0 = __float2half_rn(v0 - __half2float(h0));
+        const __half l1 = __float2half_rn(v1 - __half2float(h1));
+        hw[i] = static_cast<uint32_t>(__half_as_ushort(h0)) |
+                (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
+        lw[i] = static_cast<uint32_t>(__half_as_ushort(l0)) |
+                (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+        if (!(fabsf(v0) < 65504.f) || !(fabsf(v1) < 65504.f)) *range_bad = true;
+      }
+      const size_t at = static_cast<size_t>(unit) * D + cg * 8;
+      *reinterpret_cast<uint4*>(hi + at) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(lo + at) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
   }
 }
 

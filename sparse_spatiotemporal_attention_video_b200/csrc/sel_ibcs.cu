@@ -34,6 +34,7 @@
 // hi/lo operand splits (sel_importance.cu), fp64 sums of the softmax
 // normaliser and of the water-filling sums.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -72,10 +73,14 @@ struct KmSmem {
   int start[KM + 1];                       // first sorted position of each cluster
 };
 
+// The centroids are written as the fp16 pair hi = fp16(c), lo = fp16(c - hi),
+// the tensor-core operands of the importance scores (a centroid beyond the
+// fp16 range raises STA_DEV_RANGE).
 template <int KM>
 __global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 4 : 6) kmeans_kernel(
     const __nv_bfloat16* __restrict__ q, int N, int B, int nqb, int iters,
-    float* __restrict__ cent, float* __restrict__ wts) {
+    __half* __restrict__ cent_hi, __half* __restrict__ cent_lo, float* __restrict__ wts,
+    int32_t* dev_status) {
   constexpr int D = 128;
   extern __shared__ __align__(16) uint8_t km_raw[];
   KmSmem<KM>& sm = *reinterpret_cast<KmSmem<KM>*>(km_raw);
@@ -184,8 +189,16 @@ __global__ void __launch_bounds__(kKmThreads, KM >= 8 ? 4 : 6) kmeans_kernel(
     }
     __syncthreads();
   }
-  float* co = cent + static_cast<size_t>(row) * KM * D;
-  for (int i = tid; i < KM * D; i += kKmThreads) co[i] = -sm.negc[i];
+  const size_t co = static_cast<size_t>(row) * KM * D;
+  bool bad = false;
+  for (int i = tid; i < KM * D; i += kKmThreads) {
+    const float v = -sm.negc[i];
+    const __half h = __float2half_rn(v);
+    cent_hi[co + i] = h;
+    cent_lo[co + i] = __float2half_rn(v - __half2float(h));
+    if (!(fabsf(v) < 65504.f)) bad = true;
+  }
+  if (bad) raise_status(dev_status, STA_DEV_RANGE);
   if (tid < KM) {
     const int n = iters > 0 ? sm.start[tid + 1] - sm.start[tid] : 0;
     wts[static_cast<size_t>(row) * KM + tid] = static_cast<float>(n) / static_cast<float>(nb);
@@ -446,13 +459,15 @@ __global__ void __launch_bounds__(kSipThreads, G <= 8 ? 4 : 1) sip_sample_kernel
 }
 
 template <int KM>
-cudaError_t launch_kmeans_t(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
-                            int B, int iters, cudaStream_t s) {
+cudaError_t launch_kmeans_t(const __nv_bfloat16* q, __half* cent_hi, __half* cent_lo, float* wts,
+                            int heads, int N, int B, int iters, int32_t* dev_status,
+                            cudaStream_t s) {
   const int nqb = (N + B - 1) / B;
   const int smem = static_cast<int>(sizeof(KmSmem<KM>));
   cudaError_t e = set_dyn_smem<kmeans_kernel<KM>>(smem);
   if (e != cudaSuccess) return e;
-  kmeans_kernel<KM><<<heads * nqb, kKmThreads, smem, s>>>(q, N, B, nqb, iters, cent, wts);
+  kmeans_kernel<KM><<<heads * nqb, kKmThreads, smem, s>>>(q, N, B, nqb, iters, cent_hi, cent_lo,
+                                                          wts, dev_status);
   return cudaGetLastError();
 }
 
@@ -462,10 +477,12 @@ cudaError_t launch_kmeans_t(const __nv_bfloat16* q, float* cent, float* wts, int
 // groups per thread.
 int ibcs_max_subblocks() { return 4 * 40 * kSipThreads; }
 
-cudaError_t launch_kmeans(const __nv_bfloat16* q, float* cent, float* wts, int heads, int N,
-                          int d, int B, int km_k, int iters, cudaStream_t s) {
-#define STA_KM_CASE(KK) \
-  if (km_k == KK) return launch_kmeans_t<KK>(q, cent, wts, heads, N, B, iters, s);
+cudaError_t launch_kmeans(const __nv_bfloat16* q, __half* cent_hi, __half* cent_lo, float* wts,
+                          int heads, int N, int d, int B, int km_k, int iters,
+                          int32_t* dev_status, cudaStream_t s) {
+#define STA_KM_CASE(KK)                                                                    \
+  if (km_k == KK)                                                                          \
+    return launch_kmeans_t<KK>(q, cent_hi, cent_lo, wts, heads, N, B, iters, dev_status, s);
   if (d != 128 || B < 1 || B > kKmRows) return cudaErrorInvalidValue;
   STA_KM_CASE(4)
   STA_KM_CASE(2)

@@ -9,8 +9,9 @@
 // and 16-key sub-blocks.)
 //
 // Precision.  Sampling decisions compare u_j with pi_j = min(1, lambda p_j),
-// so p must be close to fp32 accuracy.  Each fp32 operand x is split into two
-// fp16 values, x = hi + lo with hi = fp16(x) and lo = fp16(x - hi) (22
+// so p must be close to fp32 accuracy.  Each fp32 operand x (a sub-block
+// mean or a centroid) is written by its producer (block means, k-means) as
+// two fp16 values, x = hi + lo with hi = fp16(x) and lo = fp16(x - hi) (22
 // significant bits together), and every score is accumulated in fp32 on the
 // tensor cores as hi_c.hi_k + hi_c.lo_k + lo_c.hi_k (the lo.lo term is below
 // fp32 rounding).  Against fp64 this moves pi by < 3e-7 on the workload's
@@ -355,31 +356,7 @@ __global__ void __launch_bounds__(kImpTcThreads, 1)
 }
 
 // hi = fp16(x), lo = fp16(x - hi) of an fp32 array (n elements).
-__global__ void split_f16_kernel(const float* __restrict__ x, __half* __restrict__ hi,
-                                 __half* __restrict__ lo, size_t n, int32_t* dev_status) {
-  bool bad = false;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const float v = x[i];
-    const __half h = __float2half_rn(v);
-    const float hv = __half2float(h);
-    if (!(fabsf(v) < 65504.f)) bad = true;
-    hi[i] = h;
-    lo[i] = __float2half_rn(v - hv);
-  }
-  if (bad) raise_status(dev_status, STA_DEV_RANGE);
-}
-
 }  // namespace
-
-cudaError_t launch_split_f16(const float* x, __half* hi, __half* lo, size_t n,
-                             int32_t* dev_status, cudaStream_t s) {
-  if (n == 0) return cudaSuccess;
-  size_t grid = (n + 255) / 256;
-  if (grid > 148 * 16) grid = 148 * 16;
-  split_f16_kernel<<<static_cast<unsigned>(grid), 256, 0, s>>>(x, hi, lo, n, dev_status);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_importance_tc(const float* wts, float* p, int heads, int n_rows, int nqb,
                                  int km, int n_sub, int N, int U, float scale,

@@ -1,4 +1,5 @@
-// sel_pool.cu -- block means of a [heads][N][d] bf16 tensor (fp32 out).
+// sel_pool.cu -- block means of a [heads][N][d] bf16 tensor (fp32 out, or
+// the fp16 hi/lo operand pair of the importance scores).
 //
 // "Token Radius Attention for Efficient Video Generation", 2. Methodology,
 // The TRA Pipeline: the selector works on pooled query and key blocks (the
@@ -30,6 +31,18 @@ __global__ void __launch_bounds__(kPoolThreads) block_means_kernel(
                   static_cast<long long>(blockIdx.x) * PoolShape<D, U>::UPC, part);
 }
 
+// The same means as the fp16 hi/lo pair (no fp32 copy).
+template <int D, int U>
+__global__ void __launch_bounds__(kPoolThreads) block_means_f16x2_kernel(
+    const __nv_bfloat16* __restrict__ x, __half* __restrict__ hi, __half* __restrict__ lo,
+    int heads, int N, int32_t* dev_status) {
+  __shared__ float part[kPoolThreads][9];
+  bool bad = false;
+  pool_pass<D, U>(x, nullptr, heads, N, static_cast<long long>(blockIdx.x) * PoolShape<D, U>::UPC,
+                  part, hi, lo, &bad);
+  if (bad) raise_status(dev_status, STA_DEV_RANGE);
+}
+
 template <int D, int U>
 cudaError_t launch_pool_t(const __nv_bfloat16* x0, const __nv_bfloat16* x1, float* out0,
                           float* out1, int heads, int N, cudaStream_t s) {
@@ -43,7 +56,36 @@ cudaError_t launch_pool_t(const __nv_bfloat16* x0, const __nv_bfloat16* x1, floa
   return cudaGetLastError();
 }
 
+template <int D, int U>
+cudaError_t launch_pool_f16x2_t(const __nv_bfloat16* x, __half* hi, __half* lo, int heads, int N,
+                                int32_t* dev_status, cudaStream_t s) {
+  using S = PoolShape<D, U>;
+  const long long units = static_cast<long long>(heads) * ((N + U - 1) / U);
+  const long long grid = (units + S::UPC - 1) / S::UPC;
+  if (grid <= 0) return cudaSuccess;
+  if (grid > 0x7fffffffll) return cudaErrorInvalidValue;
+  block_means_f16x2_kernel<D, U><<<static_cast<unsigned>(grid), kPoolThreads, 0, s>>>(
+      x, hi, lo, heads, N, dev_status);
+  return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_block_means_f16x2(const __nv_bfloat16* x, __half* hi, __half* lo, int heads,
+                                     int N, int d, int U, int32_t* dev_status, cudaStream_t s) {
+#define STA_POOL_CASE(DD, UU) \
+  if (d == DD && U == UU) return launch_pool_f16x2_t<DD, UU>(x, hi, lo, heads, N, dev_status, s);
+  STA_POOL_CASE(128, 128)
+  STA_POOL_CASE(128, 64)
+  STA_POOL_CASE(128, 32)
+  STA_POOL_CASE(128, 16)
+  STA_POOL_CASE(64, 128)
+  STA_POOL_CASE(64, 64)
+  STA_POOL_CASE(64, 32)
+  STA_POOL_CASE(64, 16)
+#undef STA_POOL_CASE
+  return cudaErrorInvalidValue;
+}
 
 cudaError_t launch_block_means(const __nv_bfloat16* x0, const __nv_bfloat16* x1, float* out0,
                                float* out1, int heads, int N, int d, int U, cudaStream_t s) {

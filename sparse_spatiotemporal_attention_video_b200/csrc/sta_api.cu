@@ -211,10 +211,8 @@ SelWorkspace sel_workspace(const sta_problem* p, const sta_selector_params* sel)
     w.scores = take(h * nqb * nku * 4);
   } else if (sel->kind == STA_SEL_IBCS_SIP) {
     const size_t km = sel->km_k > 0 ? static_cast<size_t>(sel->km_k) : 1;
-    w.kbar = take(h * nku * d * 4);
     w.kb_hi = take(h * nku * d * 2);
     w.kb_lo = take(h * nku * d * 2);
-    w.cent = take(h * nqb * km * d * 4);
     w.c_hi = take(h * nqb * km * d * 2);
     w.c_lo = take(h * nqb * km * d * 2);
     w.wts = take(h * nqb * km * 4);
@@ -456,8 +454,6 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
           (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return STA_ERR_WORKSPACE;
       uint8_t* ws = static_cast<uint8_t*>(workspace);
-      float* kbar = reinterpret_cast<float*>(ws + w.kbar);
-      float* cent = reinterpret_cast<float*>(ws + w.cent);
       float* wts = reinterpret_cast<float*>(ws + w.wts);
       float* pbuf = reinterpret_cast<float*>(ws + w.p);
       __half* kbh = reinterpret_cast<__half*>(ws + w.kb_hi);
@@ -469,15 +465,12 @@ sta_status sta_build_blocks(const sta_problem* prob, const sta_selector_params* 
       const float scale = 1.0f / sqrtf(static_cast<float>(prob->d));
       const int nqb = (N + sel->block_q - 1) / sel->block_q;
       const int n_rows = nqb * sel->km_k;
-      const size_t nk = static_cast<size_t>(prob->heads) * n_sub * prob->d;
-      const size_t nc = static_cast<size_t>(prob->heads) * n_rows * prob->d;
-      // 1. sub-block means, 2. k-means, 3. fp16 hi/lo splits
-      if (failed(launch_block_means(static_cast<const __nv_bfloat16*>(k), nullptr, kbar, nullptr,
-                                    prob->heads, N, prob->d, sel->kv_unit, s)) ||
-          failed(launch_kmeans(static_cast<const __nv_bfloat16*>(q), cent, wts, prob->heads, N,
-                               prob->d, sel->block_q, sel->km_k, sel->km_iters, s)) ||
-          failed(launch_split_f16(kbar, kbh, kbl, nk, dev_status, s)) ||
-          failed(launch_split_f16(cent, ch, cl, nc, dev_status, s)))
+      // 1. sub-block means, 2. k-means, both written as fp16 hi/lo pairs
+      if (failed(launch_block_means_f16x2(static_cast<const __nv_bfloat16*>(k), kbh, kbl,
+                                          prob->heads, N, prob->d, sel->kv_unit, dev_status,
+                                          s)) ||
+          failed(launch_kmeans(static_cast<const __nv_bfloat16*>(q), ch, cl, wts, prob->heads, N,
+                               prob->d, sel->block_q, sel->km_k, sel->km_iters, dev_status, s)))
         return STA_ERR_CUDA;
       // 4. importance on the tensor cores, 5. water filling + Philox sampling
       CUtensorMap tch, tcl, tkh, tkl;
