@@ -57,8 +57,8 @@ L2_FLUSH_BYTES = 256 * 1024 * 1024
 # source it was taken on (sha256 of attn_fwd.cu, first 16 hex).  Captured on
 # 2 of the 24 heads (one launch, inputs larger than L2) and scaled by 12:
 # every head carries the same work.
-NCU_TRAFFIC = {"ab_sampled": {"source_sha": "9af626cd5e3bea6c",
-                              "bytes_per_launch": 12 * (439706880 + 70045184)}}
+NCU_TRAFFIC = {"ab_sampled": {"source_sha": "90414ec2ef9bfaba",
+                              "bytes_per_launch": 12 * (422881536 + 62861056)}}
 
 
 def parse(argv=None):
