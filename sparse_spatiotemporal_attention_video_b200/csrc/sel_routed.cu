@@ -18,7 +18,7 @@
 // key T of the n_routed-th largest score and how many tokens equal to T are
 // still needed; a final pass in token order flags every token above T and
 // the first `need` tokens equal to T, and compacts the flagged ids
-// (ascending) with a block-wide scan.
+// (ascending) with block-wide scans (8 consecutive tokens per thread).
 //
 // routed_local_lists_kernel: for each query block, the kv units (kv_unit
 // consecutive tokens) holding at least one key inside the window of at least
@@ -39,6 +39,7 @@ namespace {
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelPer = 8;  // tokens per thread in the final pass
 
 // Order-preserving map fp32 -> uint32 (larger float -> larger key); -0 and
 // +0 map to the same key.
@@ -116,20 +117,42 @@ __global__ void __launch_bounds__(kSelThreads) routed_select_kernel(
   const uint32_t T = s_prefix;
   const int need_eq = s_need;  // tokens equal to T still to take (lowest ids)
   const bool none = n_routed <= 0;
+  // Final pass in token order, kSelPer consecutive tokens per thread (two
+  // block scans per kSelThreads * kSelPer tokens): the eq tokens before this
+  // thread's run decide which of its own eq tokens are taken.
   int eq_before = 0, out_before = 0;
-  for (int base = 0; base < N; base += kSelThreads) {
-    const int i = base + threadIdx.x;
-    uint32_t k = 0;
-    if (i < N) k = order_key(__ldg(dif + i));
-    const int is_eq = (i < N && k == T) ? 1 : 0;
+  for (int base = 0; base < N; base += kSelThreads * kSelPer) {
+    const int i0 = base + threadIdx.x * kSelPer;
+    uint32_t k[kSelPer];
+    int n_eq = 0;
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+      k[j] = (i0 + j < N) ? order_key(__ldg(dif + i0 + j)) : 0u;
+      n_eq += (i0 + j < N && k[j] == T) ? 1 : 0;
+    }
     int eq_excl;
-    const int eq_tot = block_exclusive_scan(is_eq, warp_tot, eq_excl);
-    const bool take = !none && i < N && (k > T || (is_eq && eq_before + eq_excl < need_eq));
+    const int eq_tot = block_exclusive_scan(n_eq, warp_tot, eq_excl);
+    int eq_seen = eq_before + eq_excl;
+    uint32_t take_bits = 0;
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+      if (i0 + j >= N || none) continue;
+      bool take = k[j] > T;
+      if (k[j] == T) {
+        take = eq_seen < need_eq;
+        ++eq_seen;
+      }
+      if (take) take_bits |= 1u << j;
+    }
     int out_excl;
-    const int out_tot = block_exclusive_scan(take ? 1 : 0, warp_tot, out_excl);
-    if (i < N) {
-      routed_flag[i] = take ? 1 : 0;
-      if (take) routed_ids[out_before + out_excl] = i;
+    const int out_tot = block_exclusive_scan(__popc(take_bits), warp_tot, out_excl);
+    int pos = out_before + out_excl;
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+      if (i0 + j >= N) continue;
+      const bool take = (take_bits >> j) & 1u;
+      routed_flag[i0 + j] = take ? 1 : 0;
+      if (take) routed_ids[pos++] = i0 + j;
     }
     eq_before += eq_tot;
     out_before += out_tot;
